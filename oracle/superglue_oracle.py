@@ -1,0 +1,289 @@
+"""Float64 CPU oracle of the SuperGlue matcher forward pass.
+
+TEST INFRASTRUCTURE ONLY.  This module is the plain, slow, step-by-step
+definition that the CUDA path is checked against.  Only the tests, the smoke
+check and the benchmark's CPU-baseline leg may import it; the library itself
+never does, and it shares no code, table or helper with the CUDA sources.
+
+Every step is written in float64 NumPy in the order and notation of the pages:
+
+* keypoint normalisation: "SuperGlue_Code_Learning / SuperGlue_model_forward_learning"
+  (Jazihars notes), the ``normalize_keypoints`` walkthrough;
+* keypoint encoder x = d + MLP_enc(x, y, c): "笔记：SuperGlue:Learning Feature
+  Matching with Graph Neural Networks论文阅读" (realcat notes), section 特征点Encode;
+  "SuperGlue 的注意力图神经网络怎样传递信息" (huluoboge blog), section
+  SuperGlue 的两类边分别带来什么;
+* attention q/k/v, softmax(q.k/sqrt(d_head)), message = sum alpha v: huluoboge
+  blog, section Attention 让节点自己选择消息来源; realcat notes, section
+  Attentional Aggregation;
+* residual update x <- x + MLP([x || m]) with self/cross alternation: realcat
+  notes, section 多层GNN; huluoboge blog, section 多轮消息怎样回到同一幅图;
+* final projection, score S = <f_A, f_B> / sqrt(D): realcat notes, section
+  匹配层 / 匹配得分预测; Jazihars notes, forward() walkthrough (score scaling);
+* dustbin augmentation and marginals a = [1_M; N], b = [1_N; M]: realcat notes,
+  section 遮挡以及可见性;
+* log-domain Sinkhorn: realcat notes, section Sinkhorn Algorithm (the author's
+  log-space optimal transport);
+* mutual nearest neighbour extraction with threshold: Jazihars notes,
+  forward() walkthrough (matches / matching scores).
+
+Readings of points the pages leave open (each is also listed in the design
+notes): BatchNorm eps = 1e-5; head h uses channels [64h, 64h+64); the heads are
+merged by a 256->256 linear layer with bias; argmax ties go to the lowest index.
+
+Parity status: see the header of each function ("pinned by" lines name the
+test that pins it).
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+F64 = np.float64
+
+
+def _as64(a):
+    return np.asarray(a, dtype=F64)
+
+
+# --------------------------------------------------------------------------- boundary
+def normalize_keypoints(kpts, width, height, mode=0):
+    """(kpt - (W/2, H/2)) / (0.7 * max(W, H))   [Jazihars notes, normalize_keypoints].
+
+    mode 1 divides by max(W, H)/2 instead (a long-side [-1, 1] normalisation).
+    Pinned by: the printed input/output values of the notes (tests/golden).
+    """
+    k = _as64(kpts)
+    center = np.array([width / 2.0, height / 2.0], F64)
+    if mode == 0:
+        scaling = max(width, height) * 0.7
+    else:
+        scaling = max(width, height) / 2.0
+    return (k - center) / scaling
+
+
+# --------------------------------------------------------------------------- MLP blocks
+def batchnorm_eval(z, gamma, beta, mean, var, eps):
+    """Eval-mode BatchNorm1d per channel: gamma (z - mean) / sqrt(var + eps) + beta.
+
+    z is (points, channels).  Pinned by: torch.nn.BatchNorm1d in eval mode.
+    """
+    return _as64(gamma) * (z - _as64(mean)) / np.sqrt(_as64(var) + eps) + _as64(beta)
+
+
+def linear(z, W, b):
+    """Kernel-size-1 Conv1d on point-major data: z (n, c_in) -> z W^T + b."""
+    out = z @ _as64(W).T
+    if b is not None:
+        out = out + _as64(b)
+    return out
+
+
+def mlp(z, Ws, bs, bns, eps):
+    """Conv1d(k=1) layers; BatchNorm + ReLU after every layer except the last
+    [realcat notes, section 特征点Encode, the MLP builder].
+    Pinned by: torch Conv1d/BatchNorm1d/ReLU Sequential with the same weights."""
+    n = len(Ws)
+    for l in range(n):
+        z = linear(z, Ws[l], bs[l])
+        if l < n - 1:
+            z = batchnorm_eval(z, *bns[l], eps)
+            z = np.maximum(z, 0.0)
+    return z
+
+
+def keypoint_encoder(kpts_norm, conf, desc, weights, eps):
+    """x0 = d + MLP_enc([x, y, c]), MLP channels 3-32-64-128-256-256, last bias 0
+    [realcat notes, section 特征点Encode; huluoboge blog, x^(0) = d + MLP_enc(p)].
+    Input order (x, y, c): keypoints first, then the confidence."""
+    p = np.concatenate([_as64(kpts_norm), _as64(conf)[:, None]], axis=1)
+    enc = mlp(p, weights["enc_W"], weights["enc_b"], weights["enc_bn"], eps)
+    return _as64(desc) + enc
+
+
+# --------------------------------------------------------------------------- attention
+def softmax(e, axis=-1):
+    """exp(e) / sum exp(e), max-shifted.  Pinned by the worked example of the
+    huluoboge blog (scores [2, 1, 0])."""
+    e = _as64(e)
+    m = np.max(e, axis=axis, keepdims=True)
+    x = np.exp(e - m)
+    return x / np.sum(x, axis=axis, keepdims=True)
+
+
+def attend(q, k, v):
+    """One head: alpha_ij = softmax_j(q_i . k_j / sqrt(d_k)); m_i = sum_j alpha_ij v_j
+    [huluoboge blog, section Attention 让节点自己选择消息来源].
+    Returns (message, alpha)."""
+    dk = q.shape[-1]
+    e = (q @ k.T) / math.sqrt(dk)
+    alpha = softmax(e, axis=1)
+    return alpha @ v, alpha
+
+
+def multi_head_attention(x, src, st, heads):
+    """q = Wq x + bq (query image), k = Wk s + bk, v = Wv s + bv (source image);
+    head h reads channels [dh*h, dh*(h+1)); the concatenated heads go through the
+    merge layer Wm, bm [realcat notes, section Attentional Aggregation].
+    Pinned by: torch.nn.MultiheadAttention with the same projections."""
+    q = linear(x, st["Wq"], st["bq"])
+    k = linear(src, st["Wk"], st["bk"])
+    v = linear(src, st["Wv"], st["bv"])
+    d = q.shape[1]
+    dh = d // heads
+    msg = np.empty((x.shape[0], d), F64)
+    for h in range(heads):
+        sl = slice(h * dh, (h + 1) * dh)
+        msg[:, sl], _ = attend(q[:, sl], k[:, sl], v[:, sl])
+    return linear(msg, st["Wm"], st["bm"])
+
+
+def attentional_propagation(x, src, st, heads, eps):
+    """delta = MLP([x || message]), MLP 512-512-256 with BN+ReLU in the middle
+    and last bias 0 [realcat notes, section 多层GNN, AttentionalPropagation]."""
+    m = multi_head_attention(x, src, st, heads)
+    z = np.concatenate([x, m], axis=1)
+    return mlp(z, [st["W1"], st["W2"]], [st["b1"], st["b2"]], [st["bn1"]], eps)
+
+
+def stage_names(n_stages):
+    """['self', 'cross'] repeated: self first [realcat notes, section 多层GNN]."""
+    return ["self" if s % 2 == 0 else "cross" for s in range(n_stages)]
+
+
+def attentional_gnn(x0, x1, weights, heads, eps, n_stages=None):
+    """Stages alternate self (A<-A, B<-B) and cross (A<-B, B<-A); both deltas are
+    computed from the pre-stage states and then added [realcat notes, section
+    多层GNN, AttentionalGNN]."""
+    stages = weights["stages"]
+    if n_stages is None:
+        n_stages = len(stages)
+    for s, name in enumerate(stage_names(n_stages)):
+        if name == "cross":
+            src0, src1 = x1, x0
+        else:
+            src0, src1 = x0, x1
+        d0 = attentional_propagation(x0, src0, stages[s], heads, eps)
+        d1 = attentional_propagation(x1, src1, stages[s], heads, eps)
+        x0, x1 = x0 + d0, x1 + d1
+    return x0, x1
+
+
+# --------------------------------------------------------------------------- matching layer
+def score_matrix(x0, x1, Wf, bf):
+    """f = Wf x + bf for both images; S_ij = <f_i^A, f_j^B> / sqrt(D)
+    [realcat notes, section 匹配得分预测; Jazihars notes, forward(), scaling by
+    descriptor_dim ** 0.5]."""
+    f0 = linear(x0, Wf, bf)
+    f1 = linear(x1, Wf, bf)
+    return (f0 @ f1.T) / math.sqrt(f0.shape[1])
+
+
+def augment_dustbin(S, alpha):
+    """S_bar = [[S, alpha 1], [alpha 1^T, alpha]] [realcat notes, section 遮挡以及可见性]."""
+    M, N = S.shape
+    Z = np.full((M + 1, N + 1), float(alpha), F64)
+    Z[:M, :N] = S
+    return Z
+
+
+def logsumexp(x, axis):
+    """log sum exp along an axis, max-shifted (all entries are finite here)."""
+    m = np.max(x, axis=axis, keepdims=True)
+    return np.squeeze(m, axis=axis) + np.log(np.sum(np.exp(x - m), axis=axis))
+
+
+def log_marginals(M, N):
+    """log mu = [norm]*M ++ [log N + norm], log nu = [norm]*N ++ [log M + norm],
+    norm = -log(M + N): the marginals a = [1_M; N], b = [1_N; M] divided by M+N
+    [realcat notes, sections 遮挡以及可见性 and Sinkhorn Algorithm]."""
+    norm = -math.log(M + N)
+    log_mu = np.full(M + 1, norm, F64)
+    log_mu[M] = math.log(N) + norm
+    log_nu = np.full(N + 1, norm, F64)
+    log_nu[N] = math.log(M) + norm
+    return log_mu, log_nu, norm
+
+
+def log_sinkhorn(Z, log_mu, log_nu, iters):
+    """u = v = 0; repeat: u = log mu - LSE_j(Z + v); v = log nu - LSE_i(Z + u).
+    Returns Z + u + v [realcat notes, section Sinkhorn Algorithm].
+    Pinned by: the 1x1 closed form, the constant-score closed form, the exact
+    column marginals, and brute-force optimal partial assignments."""
+    u = np.zeros(Z.shape[0], F64)
+    v = np.zeros(Z.shape[1], F64)
+    for _ in range(iters):
+        u = log_mu - logsumexp(Z + v[None, :], axis=1)
+        v = log_nu - logsumexp(Z + u[:, None], axis=0)
+    return Z + u[:, None] + v[None, :]
+
+
+def log_optimal_transport(S, alpha, iters):
+    """Dustbin-augmented log-domain optimal transport; the result is multiplied
+    by M + N (i.e. -norm added) so that its marginals are a and b."""
+    M, N = S.shape
+    Z = augment_dustbin(S, alpha)
+    log_mu, log_nu, norm = log_marginals(M, N)
+    return log_sinkhorn(Z, log_mu, log_nu, iters) - norm
+
+
+def extract_matches(logP, threshold):
+    """Mutual nearest neighbours on the real block of log P_bar [Jazihars notes,
+    forward(), "Get the matches with score above match_threshold"]:
+    idx0 = argmax_j, idx1 = argmax_i (lowest index on ties); mutual0_i iff
+    idx1[idx0[i]] == i; mscore0 = exp(max0) if mutual0 else 0; mscore1_j =
+    mscore0[idx1_j] if mutual1 else 0; valid0 = mutual0 and mscore0 > threshold;
+    valid1 = mutual1 and valid0[idx1_j]; invalid entries are -1.
+    Pinned by: hand-built matrices (ties, dustbin-best rows, non-mutual pairs,
+    values at the threshold)."""
+    P = _as64(logP)[:-1, :-1]
+    M, N = P.shape
+    idx0 = np.argmax(P, axis=1)          # numpy argmax returns the first maximum
+    idx1 = np.argmax(P, axis=0)
+    max0 = P[np.arange(M), idx0]
+    mutual0 = idx1[idx0] == np.arange(M)
+    mutual1 = idx0[idx1] == np.arange(N)
+    mscores0 = np.where(mutual0, np.exp(max0), 0.0)
+    mscores1 = np.where(mutual1, mscores0[idx1], 0.0)
+    valid0 = mutual0 & (mscores0 > threshold)
+    valid1 = mutual1 & valid0[idx1]
+    matches0 = np.where(valid0, idx0, -1).astype(np.int32)
+    matches1 = np.where(valid1, idx1, -1).astype(np.int32)
+    return matches0, matches1, mscores0, mscores1
+
+
+# --------------------------------------------------------------------------- whole pass
+def superglue_pair(kpts0, conf0, desc0, kpts1, conf1, desc1, weights,
+                   img_w=640.0, img_h=480.0, heads=4, iters=100,
+                   threshold=0.2, eps=1e-5, norm_mode=0, n_stages=None):
+    """One pair through the whole matcher.  Inputs point-major: kpts (n, 2) px,
+    conf (n,), desc (n, D).  Returns a dict with log_P ((M+1) x (N+1)),
+    matches0/1, mscores0/1.
+
+    Empty input (M == 0 or N == 0): matches -1 and scores 0, no log_P
+    [Jazihars notes, forward(), the "no keypoints" early return]."""
+    M, N = len(kpts0), len(kpts1)
+    if M == 0 or N == 0:
+        return {"log_P": None,
+                "matches0": np.full(M, -1, np.int32), "matches1": np.full(N, -1, np.int32),
+                "mscores0": np.zeros(M, F64), "mscores1": np.zeros(N, F64)}
+    k0 = normalize_keypoints(kpts0, img_w, img_h, norm_mode)
+    k1 = normalize_keypoints(kpts1, img_w, img_h, norm_mode)
+    x0 = keypoint_encoder(k0, conf0, desc0, weights, eps)
+    x1 = keypoint_encoder(k1, conf1, desc1, weights, eps)
+    x0, x1 = attentional_gnn(x0, x1, weights, heads, eps, n_stages)
+    S = score_matrix(x0, x1, weights["Wf"], weights["bf"])
+    logP = log_optimal_transport(S, float(weights["bin_score"]), iters)
+    m0, m1, s0, s1 = extract_matches(logP, threshold)
+    return {"log_P": logP, "matches0": m0, "matches1": m1, "mscores0": s0, "mscores1": s1,
+            "scores": S}
+
+
+def superglue_batch(batch, weights, pairs=None, **kw):
+    """Run superglue_pair on the pairs of a stacked batch (all, or a subset)."""
+    B = batch["kpts0"].shape[0]
+    idx = range(B) if pairs is None else pairs
+    return [superglue_pair(batch["kpts0"][b], batch["conf0"][b], batch["desc0"][b],
+                           batch["kpts1"][b], batch["conf1"][b], batch["desc1"][b],
+                           weights, **kw) for b in idx]

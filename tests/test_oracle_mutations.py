@@ -1,0 +1,210 @@
+"""Plant plausible mistakes in the oracle (on the CPU) and check that at least one
+pin catches each of them.  This is what makes the pins evidence: a dropped term,
+a wrong sign or index, a swapped operand anywhere in the oracle must fail one."""
+import math
+
+import numpy as np
+import pytest
+
+import test_oracle_pins as pins
+from oracle import superglue_oracle as O
+
+_extract_matches = O.extract_matches
+
+PIN_TESTS = [
+    (pins.test_normalize_keypoints_printed_values, False),
+    (pins.test_attention_worked_example, False),
+    (pins.test_attention_scale_uses_key_width, False),
+    (pins.test_batchnorm_matches_torch, True),
+    (pins.test_encoder_mlp_matches_torch_modules, True),
+    (pins.test_keypoint_encoder_adds_descriptor, True),
+    (pins.test_multi_head_attention_matches_torch, True),
+    (pins.test_attentional_propagation_matches_torch, True),
+    (pins.test_self_stage_reads_only_own_image, True),
+    (pins.test_cross_stage_reads_other_image, True),
+    (pins.test_gnn_is_symmetric_in_the_two_images, True),
+    (pins.test_cross_stage_equals_self_stage_on_the_other_source, True),
+    (pins.test_marginals_sum_to_one, False),
+    (lambda: pins.test_sinkhorn_one_by_one_closed_form(3.0, 1.0), False),
+    (lambda: pins.test_sinkhorn_constant_scores_closed_form(7), False),
+    (pins.test_sinkhorn_column_marginals_exact_and_rows_converge, False),
+    (pins.test_extraction_hand_built, False),
+    (pins.test_extraction_ties_take_lowest_index_and_threshold_is_strict, False),
+    (pins.test_score_matrix_scale_matches_library_attention, True),
+]
+
+
+def _some_pin_fails(weights):
+    for fn, needs_w in PIN_TESTS:
+        try:
+            fn(weights) if needs_w else fn()
+        except (AssertionError, ValueError, IndexError):
+            return True
+    return False
+
+
+def _attend_wrong_scale(q, k, v):
+    e = (q @ k.T) / math.sqrt(4 * q.shape[-1])
+    a = O.softmax(e, axis=1)
+    return a @ v, a
+
+
+def _attend_wrong_axis(q, k, v):
+    e = (q @ k.T) / math.sqrt(q.shape[-1])
+    a = O.softmax(e, axis=0)
+    return a @ v, a
+
+
+def _bn_eps_outside(z, g, b, m, v, eps):
+    return np.asarray(g, float) * (z - m) / (np.sqrt(np.asarray(v, float)) + eps) + b
+
+
+def _mlp_relu_before_bn(z, Ws, bs, bns, eps):
+    n = len(Ws)
+    for l in range(n):
+        z = O.linear(z, Ws[l], bs[l])
+        if l < n - 1:
+            z = np.maximum(z, 0.0)
+            z = O.batchnorm_eval(z, *bns[l], eps)
+    return z
+
+
+def _gnn_cross_uses_self(x0, x1, weights, heads, eps, n_stages=None):
+    st = weights["stages"]
+    n_stages = len(st) if n_stages is None else n_stages
+    for s in range(n_stages):
+        d0 = O.attentional_propagation(x0, x0, st[s], heads, eps)
+        d1 = O.attentional_propagation(x1, x1, st[s], heads, eps)
+        x0, x1 = x0 + d0, x1 + d1
+    return x0, x1
+
+
+def _gnn_sequential_update(x0, x1, weights, heads, eps, n_stages=None):
+    st = weights["stages"]
+    n_stages = len(st) if n_stages is None else n_stages
+    for s, name in enumerate(O.stage_names(n_stages)):
+        x0 = x0 + O.attentional_propagation(x0, x1 if name == "cross" else x0, st[s], heads, eps)
+        x1 = x1 + O.attentional_propagation(x1, x0 if name == "cross" else x1, st[s], heads, eps)
+    return x0, x1
+
+
+def _gnn_cross_first(x0, x1, weights, heads, eps, n_stages=None):
+    st = weights["stages"]
+    n_stages = len(st) if n_stages is None else n_stages
+    for s in range(n_stages):
+        cross = s % 2 == 0
+        d0 = O.attentional_propagation(x0, x1 if cross else x0, st[s], heads, eps)
+        d1 = O.attentional_propagation(x1, x0 if cross else x1, st[s], heads, eps)
+        x0, x1 = x0 + d0, x1 + d1
+    return x0, x1
+
+
+def _sinkhorn_v_first(Z, log_mu, log_nu, iters):
+    u = np.zeros(Z.shape[0])
+    v = np.zeros(Z.shape[1])
+    for _ in range(iters):
+        v = log_nu - O.logsumexp(Z + u[:, None], axis=0)
+        u = log_mu - O.logsumexp(Z + v[None, :], axis=1)
+    return Z + u[:, None] + v[None, :]
+
+
+def _marginals_swapped(M, N):
+    norm = -math.log(M + N)
+    lm = np.full(M + 1, norm)
+    lm[M] = math.log(M) + norm
+    ln = np.full(N + 1, norm)
+    ln[N] = math.log(N) + norm
+    return lm, ln, norm
+
+
+def _augment_zero_corner(S, alpha):
+    Z = np.full((S.shape[0] + 1, S.shape[1] + 1), float(alpha))
+    Z[:-1, :-1] = S
+    Z[-1, -1] = 0.0
+    return Z
+
+
+def _lot_no_renorm(S, alpha, iters):
+    M, N = S.shape
+    Z = O.augment_dustbin(S, alpha)
+    lm, ln, _ = O.log_marginals(M, N)
+    return O.log_sinkhorn(Z, lm, ln, iters)
+
+
+def _extract_ge(logP, threshold):
+    P = np.asarray(logP)[:-1, :-1]
+    M, N = P.shape
+    i0, i1 = P.argmax(1), P.argmax(0)
+    mu0, mu1 = i1[i0] == np.arange(M), i0[i1] == np.arange(N)
+    s0 = np.where(mu0, np.exp(P[np.arange(M), i0]), 0.0)
+    s1 = np.where(mu1, s0[i1], 0.0)
+    v0 = mu0 & (s0 >= threshold)
+    v1 = mu1 & v0[i1]
+    return np.where(v0, i0, -1), np.where(v1, i1, -1), s0, s1
+
+
+def _extract_last_tie(logP, threshold):
+    P = np.asarray(logP)[:-1, :-1]
+    flipped = P[:, ::-1][::-1, :]
+    m0, m1, s0, s1 = _extract_matches(np.pad(flipped, ((0, 1), (0, 1))), threshold)
+    M, N = P.shape
+    m0 = np.where(m0[::-1] >= 0, N - 1 - m0[::-1], -1)
+    m1 = np.where(m1[::-1] >= 0, M - 1 - m1[::-1], -1)
+    return m0, m1, s0[::-1], s1[::-1]
+
+
+def _normalize_hw_swapped(kpts, width, height, mode=0):
+    return (np.asarray(kpts, float) - np.array([height / 2, width / 2])) / (0.7 * max(width, height))
+
+
+def _score_unscaled(x0, x1, Wf, bf):
+    return O.linear(x0, Wf, bf) @ O.linear(x1, Wf, bf).T
+
+
+def _mha_interleaved_heads(x, src, st, heads):
+    q = O.linear(x, st["Wq"], st["bq"])
+    k = O.linear(src, st["Wk"], st["bk"])
+    v = O.linear(src, st["Wv"], st["bv"])
+    msg = np.empty_like(q)
+    for h in range(heads):
+        sl = slice(h, None, heads)
+        msg[:, sl], _ = O.attend(q[:, sl], k[:, sl], v[:, sl])
+    return O.linear(msg, st["Wm"], st["bm"])
+
+
+def _prop_message_first(x, src, st, heads, eps):
+    m = O.multi_head_attention(x, src, st, heads)
+    z = np.concatenate([m, x], axis=1)
+    return O.mlp(z, [st["W1"], st["W2"]], [st["b1"], st["b2"]], [st["bn1"]], eps)
+
+
+MUTATIONS = {
+    "attention scale 1/sqrt(D)": ("attend", _attend_wrong_scale),
+    "softmax over queries": ("attend", _attend_wrong_axis),
+    "BN eps outside sqrt": ("batchnorm_eval", _bn_eps_outside),
+    "ReLU before BN": ("mlp", _mlp_relu_before_bn),
+    "cross stage reads own image": ("attentional_gnn", _gnn_cross_uses_self),
+    "sequential A-then-B update": ("attentional_gnn", _gnn_sequential_update),
+    "cross stage first": ("attentional_gnn", _gnn_cross_first),
+    "Sinkhorn column update first": ("log_sinkhorn", _sinkhorn_v_first),
+    "dustbin marginals swapped": ("log_marginals", _marginals_swapped),
+    "dustbin corner zero": ("augment_dustbin", _augment_zero_corner),
+    "missing M+N rescale": ("log_optimal_transport", _lot_no_renorm),
+    "threshold not strict": ("extract_matches", _extract_ge),
+    "ties to the last index": ("extract_matches", _extract_last_tie),
+    "width/height swapped": ("normalize_keypoints", _normalize_hw_swapped),
+    "score without 1/sqrt(D)": ("score_matrix", _score_unscaled),
+    "interleaved head channels": ("multi_head_attention", _mha_interleaved_heads),
+    "[m || x] concatenation": ("attentional_propagation", _prop_message_first),
+}
+
+
+def test_unmutated_oracle_passes_every_pin(weights):
+    assert not _some_pin_fails(weights)
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_each_planted_mistake_is_caught(name, weights, monkeypatch):
+    attr, fn = MUTATIONS[name]
+    monkeypatch.setattr(O, attr, fn)
+    assert _some_pin_fails(weights), f"no pin catches: {name}"

@@ -1,0 +1,371 @@
+"""Pins of the float64 oracle against things other than itself: values the pages
+print, library routines (torch float64 modules), closed forms, invariants and
+brute force.  CPU only."""
+import itertools
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from conftest import golden_path
+from oracle import superglue_oracle as O
+from learned_sparse_feature_b200 import synth
+
+
+def _read_golden(name):
+    rows = []
+    with open(golden_path(name)) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                rows.append(line.split())
+    return rows
+
+
+# --------------------------------------------------------------------------- printed values
+def test_normalize_keypoints_printed_values():
+    rows = np.array(_read_golden("normalize_keypoints_427x640.txt"), float)
+    out = O.normalize_keypoints(rows[:, :2], width=640.0, height=427.0, mode=0)
+    # outputs printed to 5 significant digits, inputs to 1e-4 px (/448 px)
+    tol = 5e-5 * np.abs(rows[:, 2:]) + 1.2e-7
+    assert np.all(np.abs(out - rows[:, 2:]) <= tol)
+
+
+def test_normalize_mode1_is_long_side_unit_range():
+    corners = np.array([[0.0, 0.0], [640.0, 480.0]])
+    out = O.normalize_keypoints(corners, 640.0, 480.0, mode=1)
+    np.testing.assert_allclose(out, [[-1.0, -0.75], [1.0, 0.75]], rtol=0, atol=1e-15)
+
+
+def test_attention_worked_example():
+    g = {r[0]: [float(v) for v in r[1:]] for r in _read_golden("attention_worked_example.txt")
+         if r[0] != "value"}
+    values = np.array([[float(v) for v in r[1:]] for r in _read_golden("attention_worked_example.txt")
+                       if r[0] == "value"])
+    w = O.softmax(np.array(g["scores"]))
+    np.testing.assert_allclose(w, g["weights"], atol=5e-4)
+    # same example through one attention head: d_k = 1, q = 1, k_j = score_j
+    q = np.array([[1.0]])
+    k = np.array(g["scores"])[:, None]
+    msg, alpha = O.attend(q, k, values)
+    np.testing.assert_allclose(alpha[0], g["weights"], atol=5e-4)
+    np.testing.assert_allclose(msg[0], g["message"], atol=5e-4)
+
+
+def test_attention_scale_uses_key_width():
+    # d_k = 4: q.k = 8 for the first key -> e = 8 / sqrt(4) = 4
+    q = np.array([[1.0, 1.0, 1.0, 1.0]])
+    k = np.array([[2.0, 2.0, 2.0, 2.0], [0.0, 0.0, 0.0, 0.0]])
+    _, alpha = O.attend(q, k, np.eye(2))
+    np.testing.assert_allclose(alpha[0, 0], 1.0 / (1.0 + math.exp(-4.0)), rtol=1e-14)
+
+
+# --------------------------------------------------------------------------- library pins
+def _torch_mlp(Ws, bs, bns, eps):
+    layers = []
+    n = len(Ws)
+    for l in range(n):
+        conv = torch.nn.Conv1d(Ws[l].shape[1], Ws[l].shape[0], kernel_size=1, bias=True).double()
+        conv.weight.data = torch.tensor(np.asarray(Ws[l], float))[:, :, None]
+        conv.bias.data = torch.tensor(np.asarray(bs[l], float))
+        layers.append(conv)
+        if l < n - 1:
+            bn = torch.nn.BatchNorm1d(Ws[l].shape[0], eps=eps).double()
+            g, b, m, v = (torch.tensor(np.asarray(a, float)) for a in bns[l])
+            bn.weight.data, bn.bias.data = g, b
+            bn.running_mean.data, bn.running_var.data = m, v
+            layers.append(bn)
+            layers.append(torch.nn.ReLU())
+    return torch.nn.Sequential(*layers).eval()
+
+
+def test_batchnorm_matches_torch(weights):
+    rng = np.random.default_rng(1)
+    z = rng.standard_normal((50, 32))
+    stats = weights["enc_bn"][0]
+    bn = torch.nn.BatchNorm1d(32, eps=1e-5).double().eval()
+    bn.weight.data, bn.bias.data = (torch.tensor(np.asarray(a, float)) for a in stats[:2])
+    bn.running_mean.data, bn.running_var.data = (torch.tensor(np.asarray(a, float)) for a in stats[2:])
+    with torch.no_grad():
+        ref = bn(torch.tensor(z)).numpy()
+    np.testing.assert_allclose(O.batchnorm_eval(z, *stats, 1e-5), ref, rtol=1e-13, atol=1e-13)
+
+
+def test_batchnorm_identity_stats_is_plain_scaling():
+    z = np.linspace(-3, 3, 12).reshape(4, 3)
+    one, zero = np.ones(3), np.zeros(3)
+    np.testing.assert_allclose(O.batchnorm_eval(z, one, zero, zero, one, 1e-5),
+                               z / math.sqrt(1.0 + 1e-5), rtol=1e-15)
+
+
+def test_encoder_mlp_matches_torch_modules(weights):
+    rng = np.random.default_rng(2)
+    p = rng.uniform(-0.7, 0.7, (40, 3))
+    net = _torch_mlp(weights["enc_W"], weights["enc_b"], weights["enc_bn"], 1e-5)
+    with torch.no_grad():
+        ref = net(torch.tensor(p.T[None]))[0].numpy().T      # channels-first in torch
+    out = O.mlp(p, weights["enc_W"], weights["enc_b"], weights["enc_bn"], 1e-5)
+    np.testing.assert_allclose(out, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_keypoint_encoder_adds_descriptor(weights):
+    rng = np.random.default_rng(3)
+    k = rng.uniform(-0.7, 0.7, (10, 2))
+    c = rng.uniform(0, 1, 10)
+    d = rng.standard_normal((10, 256))
+    net = _torch_mlp(weights["enc_W"], weights["enc_b"], weights["enc_bn"], 1e-5)
+    inp = torch.cat([torch.tensor(k.T[None]), torch.tensor(c[None, None])], dim=1)
+    with torch.no_grad():
+        ref = d + net(inp)[0].numpy().T
+    np.testing.assert_allclose(O.keypoint_encoder(k, c, d, weights, 1e-5), ref, rtol=1e-12, atol=1e-12)
+
+
+def _torch_mha(st, d=256, heads=4):
+    mha = torch.nn.MultiheadAttention(d, heads, bias=True, batch_first=True).double().eval()
+    W = np.concatenate([st["Wq"], st["Wk"], st["Wv"]]).astype(float)
+    b = np.concatenate([st["bq"], st["bk"], st["bv"]]).astype(float)
+    mha.in_proj_weight.data = torch.tensor(W)
+    mha.in_proj_bias.data = torch.tensor(b)
+    mha.out_proj.weight.data = torch.tensor(np.asarray(st["Wm"], float))
+    mha.out_proj.bias.data = torch.tensor(np.asarray(st["bm"], float))
+    return mha
+
+
+def test_multi_head_attention_matches_torch(weights):
+    rng = np.random.default_rng(4)
+    x = rng.standard_normal((17, 256)) * 0.3
+    src = rng.standard_normal((23, 256)) * 0.3
+    st = weights["stages"][0]
+    mha = _torch_mha(st)
+    with torch.no_grad():
+        ref, _ = mha(torch.tensor(x[None]), torch.tensor(src[None]), torch.tensor(src[None]))
+    np.testing.assert_allclose(O.multi_head_attention(x, src, st, 4), ref[0].numpy(),
+                               rtol=1e-11, atol=1e-12)
+
+
+def test_attentional_propagation_matches_torch(weights):
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((19, 256)) * 0.3
+    src = rng.standard_normal((11, 256)) * 0.3
+    st = weights["stages"][3]
+    mha = _torch_mha(st)
+    net = _torch_mlp([st["W1"], st["W2"]], [st["b1"], st["b2"]], [st["bn1"]], 1e-5)
+    with torch.no_grad():
+        m, _ = mha(torch.tensor(x[None]), torch.tensor(src[None]), torch.tensor(src[None]))
+        z = torch.cat([torch.tensor(x[None]), m], dim=2).transpose(1, 2)
+        ref = net(z)[0].numpy().T
+    np.testing.assert_allclose(O.attentional_propagation(x, src, st, 4, 1e-5), ref,
+                               rtol=1e-10, atol=1e-12)
+
+
+def test_sinkhorn_logsumexp_matches_torch():
+    rng = np.random.default_rng(6)
+    x = rng.standard_normal((7, 9)) * 30
+    np.testing.assert_allclose(O.logsumexp(x, 1), torch.logsumexp(torch.tensor(x), 1).numpy(), rtol=1e-14)
+    np.testing.assert_allclose(O.logsumexp(x, 0), torch.logsumexp(torch.tensor(x), 0).numpy(), rtol=1e-14)
+
+
+# --------------------------------------------------------------------------- GNN structure
+def _pair(n0, n1, seed):
+    rng = np.random.default_rng(seed)
+    return (rng.standard_normal((n0, 256)) * 0.3, rng.standard_normal((n1, 256)) * 0.3)
+
+
+def test_self_stage_reads_only_own_image(weights):
+    x0, x1 = _pair(9, 7, 7)
+    a0, _ = O.attentional_gnn(x0, x1, weights, 4, 1e-5, n_stages=1)
+    b0, _ = O.attentional_gnn(x0, x1 * 2.0 + 0.1, weights, 4, 1e-5, n_stages=1)
+    np.testing.assert_array_equal(a0, b0)
+
+
+def test_cross_stage_reads_other_image(weights):
+    x0, x1 = _pair(9, 7, 8)
+    a0, _ = O.attentional_gnn(x0, x1, weights, 4, 1e-5, n_stages=2)
+    b0, _ = O.attentional_gnn(x0, x1 * 2.0 + 0.1, weights, 4, 1e-5, n_stages=2)
+    assert np.abs(a0 - b0).max() > 1e-3
+
+
+def test_gnn_is_symmetric_in_the_two_images(weights):
+    # shared weights + simultaneous update: swapping the images swaps the outputs
+    x0, x1 = _pair(9, 7, 9)
+    a0, a1 = O.attentional_gnn(x0, x1, weights, 4, 1e-5, n_stages=4)
+    b1, b0 = O.attentional_gnn(x1, x0, weights, 4, 1e-5, n_stages=4)
+    np.testing.assert_allclose(a0, b0, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(a1, b1, rtol=0, atol=1e-13)
+
+
+def test_cross_stage_equals_self_stage_on_the_other_source(weights):
+    # a single cross stage on (x0, x1) gives A the delta a self stage would give
+    # a query set x0 attending to x1, i.e. attentional_propagation(x0, x1)
+    x0, x1 = _pair(6, 8, 10)
+    st = weights["stages"][1]
+    y0, y1 = O.attentional_gnn(x0, x1, {"stages": [weights["stages"][0], st]}, 4, 1e-5, n_stages=2)
+    s0, s1 = O.attentional_gnn(x0, x1, weights, 4, 1e-5, n_stages=1)
+    np.testing.assert_allclose(y0 - s0, O.attentional_propagation(s0, s1, st, 4, 1e-5), atol=1e-13)
+    np.testing.assert_allclose(y1 - s1, O.attentional_propagation(s1, s0, st, 4, 1e-5), atol=1e-13)
+
+
+# --------------------------------------------------------------------------- Sinkhorn
+def test_marginals_sum_to_one():
+    for M, N in [(1, 1), (5, 3), (64, 100)]:
+        lm, ln, norm = O.log_marginals(M, N)
+        assert abs(np.exp(lm).sum() - 1) < 1e-14 and abs(np.exp(ln).sum() - 1) < 1e-14
+        assert abs(norm + math.log(M + N)) < 1e-15
+
+
+@pytest.mark.parametrize("s,z", [(3.0, 1.0), (-2.0, 1.0), (0.5, -4.0)])
+def test_sinkhorn_one_by_one_closed_form(s, z):
+    # S_bar = [[s, z], [z, z]], all marginals 1: fixed point [[p, 1-p], [1-p, p]]
+    # with cross-ratio p^2 / (1-p)^2 = exp(s - z), i.e. p = sigmoid((s - z) / 2)
+    P = np.exp(O.log_optimal_transport(np.array([[s]]), z, iters=200))
+    p = 1.0 / (1.0 + math.exp(-(s - z) / 2.0))
+    np.testing.assert_allclose(P, [[p, 1 - p], [1 - p, p]], rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("T", [1, 7])
+def test_sinkhorn_constant_scores_closed_form(T):
+    M, N, z = 5, 3, 0.7
+    logP = O.log_optimal_transport(np.full((M, N), z), z, iters=T)
+    a = np.r_[np.ones(M), N]
+    b = np.r_[np.ones(N), M]
+    np.testing.assert_allclose(np.exp(logP), np.outer(a, b) / (M + N), rtol=1e-13)
+
+
+def test_sinkhorn_column_marginals_exact_and_rows_converge():
+    rng = np.random.default_rng(11)
+    M, N = 13, 9
+    S = rng.standard_normal((M, N)) * 3
+    a = np.r_[np.ones(M), N]
+    b = np.r_[np.ones(N), M]
+    prev = np.inf
+    for T in (1, 3, 10, 30, 100):
+        P = np.exp(O.log_optimal_transport(S, 1.0, T))
+        np.testing.assert_allclose(P.sum(0), b, rtol=1e-12)       # v is updated last
+        res = np.abs(P.sum(1) - a).max()
+        assert res <= prev + 1e-15
+        prev = res
+    assert prev < 1e-6
+
+
+def _best_partial_assignment(S, z):
+    """Brute force: the partial injection maximising sum (S_ij - z)."""
+    M, N = S.shape
+    best, arg = -np.inf, None
+    for k in range(0, min(M, N) + 1):
+        for rows in itertools.combinations(range(M), k):
+            for cols in itertools.permutations(range(N), k):
+                val = sum(S[i, j] - z for i, j in zip(rows, cols))
+                if val > best + 1e-12:
+                    best, arg = val, dict(zip(rows, cols))
+    return best, arg
+
+
+def _second_best_gap(S, z, best):
+    M, N = S.shape
+    vals = []
+    for k in range(0, min(M, N) + 1):
+        for rows in itertools.combinations(range(M), k):
+            for cols in itertools.permutations(range(N), k):
+                vals.append(sum(S[i, j] - z for i, j in zip(rows, cols)))
+    vals = np.sort(np.array(vals))[::-1]
+    return best - vals[1] if len(vals) > 1 else np.inf
+
+
+def test_sinkhorn_low_temperature_is_optimal_partial_assignment():
+    rng = np.random.default_rng(12)
+    eps, z = 0.02, 1.0
+    checked = 0
+    for trial in range(200):
+        M, N = rng.integers(1, 5), rng.integers(1, 5)
+        S = rng.uniform(-1.0, 4.0, (M, N))
+        best, assign = _best_partial_assignment(S, z)
+        if _second_best_gap(S, z, best) < 0.5:
+            continue
+        P = np.exp(O.log_optimal_transport(S / eps, z / eps, iters=3000))
+        for i in range(M):
+            j = assign.get(i, N)                       # N = dustbin column
+            assert P[i, j] > 0.95, (trial, i, j, P)
+        for j in range(N):
+            i = {c: r for r, c in assign.items()}.get(j, M)
+            assert P[i, j] > 0.95
+        checked += 1
+        if checked >= 25:
+            break
+    assert checked >= 25
+
+
+# --------------------------------------------------------------------------- extraction
+def test_extraction_hand_built():
+    thr = 0.2
+    # real block 4 x 4 (+ dustbin row/col).  Probabilities, then log.
+    P = np.full((5, 5), 1e-3)
+    P[0, 1] = 0.90      # row 0 <-> col 1 mutual, above threshold
+    P[1, 0] = 0.15      # row 1 <-> col 0 mutual, below threshold
+    P[1, 4] = 0.80      # row 1's best is the dustbin; real argmax still col 0
+    P[2, 2] = 0.50      # row 2 -> col 2, but col 2's best is row 3: not mutual
+    P[3, 2] = 0.60
+    P[3, 3] = 0.55      # row 3 -> col 2 (0.60 > 0.55); col 3 -> row 3 (not mutual for col 3)
+    P[2, 3] = 0.30
+    logP = np.log(P)
+    m0, m1, s0, s1 = O.extract_matches(logP, thr)
+    np.testing.assert_array_equal(m0, [1, -1, -1, 2])
+    np.testing.assert_array_equal(m1, [-1, 0, 3, -1])
+    np.testing.assert_allclose(s0, [0.90, 0.15, 0.0, 0.60], rtol=1e-12)
+    np.testing.assert_allclose(s1, [0.15, 0.90, 0.60, 0.0], rtol=1e-12)
+
+
+def test_extraction_ties_take_lowest_index_and_threshold_is_strict():
+    P = np.full((3, 3), 0.01)
+    P[0, 0] = P[0, 1] = 0.5     # tie in row 0 -> col 0; col 0 -> row 0 (mutual)
+    logP = np.log(P)
+    at = float(np.exp(logP[0, 0]))                   # the score row 0 will get
+    m0, m1, s0, _ = O.extract_matches(logP, at)      # exactly at threshold: rejected
+    assert m0[0] == -1 and s0[0] == at
+    m0, m1, _, _ = O.extract_matches(logP, 0.49)
+    assert m0[0] == 0 and m1[0] == 0 and m1[1] == -1
+
+
+def test_empty_input(weights):
+    r = O.superglue_pair(np.zeros((0, 2)), np.zeros(0), np.zeros((0, 256)),
+                         np.ones((3, 2)), np.ones(3), np.ones((3, 256)), weights)
+    assert r["log_P"] is None
+    np.testing.assert_array_equal(r["matches1"], [-1, -1, -1])
+    np.testing.assert_array_equal(r["mscores1"], [0, 0, 0])
+    assert r["matches0"].shape == (0,)
+
+
+# --------------------------------------------------------------------------- whole network
+def test_full_network_permutation_equivariance(weights):
+    batch = synth.make_batch("pair64_fp32")
+    k0, c0, d0 = batch["kpts0"][0], batch["conf0"][0], batch["desc0"][0]
+    k1, c1, d1 = batch["kpts1"][0][:48], batch["conf1"][0][:48], batch["desc1"][0][:48]
+    ref = O.superglue_pair(k0, c0, d0, k1, c1, d1, weights, n_stages=4)
+    rng = np.random.default_rng(13)
+    pa, pb = rng.permutation(len(k0)), rng.permutation(len(k1))
+    out = O.superglue_pair(k0[pa], c0[pa], d0[pa], k1[pb], c1[pb], d1[pb], weights, n_stages=4)
+    ra = np.r_[pa, len(k0)]
+    rb = np.r_[pb, len(k1)]
+    np.testing.assert_allclose(out["log_P"], ref["log_P"][np.ix_(ra, rb)], rtol=0, atol=1e-10)
+    inv_b = np.argsort(pb)
+    inv_a = np.argsort(pa)
+    exp0 = np.where(ref["matches0"][pa] >= 0, inv_b[np.maximum(ref["matches0"][pa], 0)], -1)
+    exp1 = np.where(ref["matches1"][pb] >= 0, inv_a[np.maximum(ref["matches1"][pb], 0)], -1)
+    np.testing.assert_array_equal(out["matches0"], exp0)
+    np.testing.assert_array_equal(out["matches1"], exp1)
+
+
+def test_score_matrix_scale_matches_library_attention(weights):
+    # softmax_j(S_ij) with S = <f_i^A, f_j^B> / sqrt(D) is exactly what the library's
+    # scaled-dot-product attention computes for q = f^A, k = f^B, v = I (default
+    # scale 1/sqrt(D)).  Softmax is shift- but not scale-invariant, so this pins
+    # the 1/sqrt(D) factor and the operand order.
+    rng = np.random.default_rng(14)
+    x0 = rng.standard_normal((6, 256)) * 0.3
+    x1 = rng.standard_normal((9, 256)) * 0.3
+    S = O.score_matrix(x0, x1, weights["Wf"], weights["bf"])
+    f0 = O.linear(x0, weights["Wf"], weights["bf"])
+    f1 = O.linear(x1, weights["Wf"], weights["bf"])
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.tensor(f0[None]), torch.tensor(f1[None]), torch.eye(9, dtype=torch.float64)[None])[0]
+    np.testing.assert_allclose(O.softmax(S, axis=1), ref.numpy(), rtol=1e-10, atol=1e-13)
