@@ -1,0 +1,233 @@
+"""Thin ctypes binding of libsg (include/sg.h).  Argument marshalling only: every
+step of the matcher runs in the library's CUDA kernels.  Torch is used for
+device memory and streams; the calls take torch tensors and pass their device
+pointers through the C ABI.
+
+The library is loaded from this package directory (built in-tree by
+``learned_sparse_feature_b200.build``); a missing library is an error, there is
+no fallback.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+import numpy as np
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libsg.so")
+
+SG_MAX_STAGES = 32
+SG_ENC_LAYERS = 5
+
+STATUS = {0: "SG_OK", 1: "SG_ERR_INVALID_ARG", 2: "SG_ERR_SHAPE", 3: "SG_ERR_OOM",
+          4: "SG_ERR_CUDA", 5: "SG_ERR_TIMEOUT", 6: "SG_ERR_NUMERIC", 7: "SG_ERR_UNSUPPORTED"}
+
+EXPORTED = ["sg_create", "sg_destroy", "sg_match", "sg_match_host", "sg_scores",
+            "sg_optimal_transport", "sg_status", "sg_strerror", "sg_launches_per_match",
+            "sg_selftest_barrier_timeout"]
+
+_FP = C.POINTER(C.c_float)
+
+
+class SgWeights(C.Structure):
+    _fields_ = [
+        ("enc_W", _FP * SG_ENC_LAYERS),
+        ("enc_b", _FP * SG_ENC_LAYERS),
+        ("enc_bn", (_FP * 4) * (SG_ENC_LAYERS - 1)),
+        ("Wq", _FP * SG_MAX_STAGES), ("bq", _FP * SG_MAX_STAGES),
+        ("Wk", _FP * SG_MAX_STAGES), ("bk", _FP * SG_MAX_STAGES),
+        ("Wv", _FP * SG_MAX_STAGES), ("bv", _FP * SG_MAX_STAGES),
+        ("Wm", _FP * SG_MAX_STAGES), ("bm", _FP * SG_MAX_STAGES),
+        ("W1", _FP * SG_MAX_STAGES), ("b1", _FP * SG_MAX_STAGES),
+        ("bn1", (_FP * 4) * SG_MAX_STAGES),
+        ("W2", _FP * SG_MAX_STAGES),
+        ("Wf", _FP), ("bf", _FP),
+        ("bin_score", C.c_float),
+    ]
+
+
+class SgConfig(C.Structure):
+    _fields_ = [
+        ("D", C.c_int), ("H", C.c_int), ("n_stages", C.c_int), ("sinkhorn_iters", C.c_int),
+        ("match_threshold", C.c_float), ("bn_eps", C.c_float), ("precision", C.c_int),
+        ("img_w", C.c_float), ("img_h", C.c_float), ("norm_mode", C.c_int),
+        ("max_B", C.c_int), ("max_M", C.c_int), ("max_N", C.c_int),
+    ]
+
+
+class SgError(RuntimeError):
+    def __init__(self, code, where):
+        super().__init__(f"{where}: {STATUS.get(code, code)}")
+        self.code = code
+
+
+_lib = None
+
+
+def load():
+    """Load libsg.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"libsg.so not built at {LIB_PATH}; run learned_sparse_feature_b200.build")
+    lib = C.CDLL(LIB_PATH)
+    vp, i32, f32 = C.c_void_p, C.c_int, C.c_float
+    lib.sg_create.argtypes = [C.POINTER(SgWeights), C.POINTER(SgConfig), C.POINTER(vp)]
+    lib.sg_create.restype = i32
+    lib.sg_destroy.argtypes = [vp]
+    lib.sg_destroy.restype = None
+    io = [vp, i32, i32, i32, vp, vp, vp, vp, vp, vp]
+    lib.sg_match.argtypes = io + [vp, vp, vp, vp, vp, vp]
+    lib.sg_match.restype = i32
+    lib.sg_match_host.argtypes = io + [vp, vp, vp, vp, vp, vp]
+    lib.sg_match_host.restype = i32
+    lib.sg_scores.argtypes = io + [vp, vp]
+    lib.sg_scores.restype = i32
+    lib.sg_optimal_transport.argtypes = [vp, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp]
+    lib.sg_optimal_transport.restype = i32
+    lib.sg_status.argtypes = [vp, vp]
+    lib.sg_status.restype = i32
+    lib.sg_strerror.argtypes = [i32]
+    lib.sg_strerror.restype = C.c_char_p
+    lib.sg_launches_per_match.argtypes = [vp, i32, i32, i32]
+    lib.sg_launches_per_match.restype = i32
+    lib.sg_selftest_barrier_timeout.argtypes = [vp, C.c_uint, vp]
+    lib.sg_selftest_barrier_timeout.restype = i32
+    _lib = lib
+    return lib
+
+
+def _check(code, where):
+    if code != 0:
+        raise SgError(code, where)
+
+
+def _ptr(t):
+    """Device (or host) pointer of a torch tensor / numpy array, or None."""
+    if t is None:
+        return None
+    if isinstance(t, np.ndarray):
+        return t.ctypes.data
+    return t.data_ptr()
+
+
+def _stream_ptr(stream):
+    if stream is None:
+        import torch
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+class Matcher:
+    """A libsg handle: packed weights plus a workspace for (max_B, max_M, max_N)."""
+
+    def __init__(self, weights: dict, max_B: int, max_M: int, max_N: int, precision: str = "bf16",
+                 n_stages: int | None = None, sinkhorn_iters: int = 100, match_threshold: float = 0.2,
+                 bn_eps: float = 1e-5, img_w: float = 640.0, img_h: float = 480.0, norm_mode: int = 0):
+        lib = load()
+        self._keep = []
+        w = SgWeights()
+
+        def fp(a):
+            a = np.ascontiguousarray(np.asarray(a, np.float32))
+            self._keep.append(a)
+            return a.ctypes.data_as(_FP)
+
+        for l in range(SG_ENC_LAYERS):
+            w.enc_W[l] = fp(weights["enc_W"][l])
+            w.enc_b[l] = fp(weights["enc_b"][l])
+            if l < SG_ENC_LAYERS - 1:
+                for k in range(4):
+                    w.enc_bn[l][k] = fp(weights["enc_bn"][l][k])
+        stages = weights["stages"]
+        n = len(stages) if n_stages is None else n_stages
+        for s in range(n):
+            st = stages[s]
+            for nm in ("Wq", "bq", "Wk", "bk", "Wv", "bv", "Wm", "bm", "W1", "b1", "W2"):
+                getattr(w, nm)[s] = fp(st[nm])
+            for k in range(4):
+                w.bn1[s][k] = fp(st["bn1"][k])
+        w.Wf = fp(weights["Wf"])
+        w.bf = fp(weights["bf"])
+        w.bin_score = float(weights["bin_score"])
+        cfg = SgConfig(256, 4, n, sinkhorn_iters, match_threshold, bn_eps,
+                       1 if precision == "bf16" else 0, img_w, img_h, norm_mode, max_B, max_M, max_N)
+        h = C.c_void_p()
+        _check(lib.sg_create(C.byref(w), C.byref(cfg), C.byref(h)), "sg_create")
+        self._keep = []
+        self.h = h
+        self.lib = lib
+        self.cfg = cfg
+
+    def close(self):
+        if getattr(self, "h", None):
+            self.lib.sg_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    # -- device API -----------------------------------------------------------------
+    def match(self, kpts0, conf0, desc0, kpts1, conf1, desc1, out_logP, matches0, matches1,
+              mscores0, mscores1, stream=None):
+        B, M, N = kpts0.shape[0], kpts0.shape[1], kpts1.shape[1]
+        _check(self.lib.sg_match(self.h, B, M, N, _ptr(kpts0), _ptr(conf0), _ptr(desc0), _ptr(kpts1),
+                                 _ptr(conf1), _ptr(desc1), _ptr(out_logP), _ptr(matches0),
+                                 _ptr(matches1), _ptr(mscores0), _ptr(mscores1), _stream_ptr(stream)),
+               "sg_match")
+
+    def match_host(self, kpts0, conf0, desc0, kpts1, conf1, desc1, out_logP, matches0, matches1,
+                   mscores0, mscores1, stream=None):
+        B, M, N = kpts0.shape[0], kpts0.shape[1], kpts1.shape[1]
+        _check(self.lib.sg_match_host(self.h, B, M, N, _ptr(kpts0), _ptr(conf0), _ptr(desc0),
+                                      _ptr(kpts1), _ptr(conf1), _ptr(desc1), _ptr(out_logP),
+                                      _ptr(matches0), _ptr(matches1), _ptr(mscores0), _ptr(mscores1),
+                                      _stream_ptr(stream)), "sg_match_host")
+
+    def scores(self, kpts0, conf0, desc0, kpts1, conf1, desc1, out_scores, stream=None):
+        B, M, N = kpts0.shape[0], kpts0.shape[1], kpts1.shape[1]
+        _check(self.lib.sg_scores(self.h, B, M, N, _ptr(kpts0), _ptr(conf0), _ptr(desc0), _ptr(kpts1),
+                                  _ptr(conf1), _ptr(desc1), _ptr(out_scores), _stream_ptr(stream)),
+               "sg_scores")
+
+    def optimal_transport(self, scores, out_logP, matches0, matches1, mscores0, mscores1, stream=None):
+        B, M, N = scores.shape
+        _check(self.lib.sg_optimal_transport(self.h, B, M, N, _ptr(scores), _ptr(out_logP),
+                                             _ptr(matches0), _ptr(matches1), _ptr(mscores0),
+                                             _ptr(mscores1), _stream_ptr(stream)),
+               "sg_optimal_transport")
+
+    def status(self, stream=None):
+        return self.lib.sg_status(self.h, _stream_ptr(stream))
+
+    def selftest_barrier_timeout(self, timeout_us=20000, stream=None):
+        return self.lib.sg_selftest_barrier_timeout(self.h, timeout_us, _stream_ptr(stream))
+
+    def launches_per_match(self, B, M, N):
+        return self.lib.sg_launches_per_match(self.h, B, M, N)
+
+
+def match_batch(matcher: Matcher, batch: dict, with_logP: bool = True, stream=None):
+    """Convenience: run sg_match on a synthetic batch (numpy) and return numpy outputs."""
+    import torch
+    dev = torch.device("cuda")
+    t = {k: torch.from_numpy(np.ascontiguousarray(batch[k])).to(dev)
+         for k in ("kpts0", "conf0", "desc0", "kpts1", "conf1", "desc1")}
+    B, M, N = batch["kpts0"].shape[0], batch["kpts0"].shape[1], batch["kpts1"].shape[1]
+    logP = torch.empty((B, M + 1, N + 1), dtype=torch.float32, device=dev) if with_logP else None
+    m0 = torch.empty((B, M), dtype=torch.int32, device=dev)
+    m1 = torch.empty((B, N), dtype=torch.int32, device=dev)
+    s0 = torch.empty((B, M), dtype=torch.float32, device=dev)
+    s1 = torch.empty((B, N), dtype=torch.float32, device=dev)
+    matcher.match(t["kpts0"], t["conf0"], t["desc0"], t["kpts1"], t["conf1"], t["desc1"],
+                  logP, m0, m1, s0, s1, stream)
+    _check(matcher.status(stream), "device status")
+    out = {"matches0": m0.cpu().numpy(), "matches1": m1.cpu().numpy(),
+           "mscores0": s0.cpu().numpy(), "mscores1": s1.cpu().numpy()}
+    out["log_P"] = logP.cpu().numpy() if with_logP else None
+    return out

@@ -1,0 +1,625 @@
+// Host side of libsg: the C ABI, weight folding/packing, workspace planning and
+// the launch sequence of one forward pass (optionally replayed as a CUDA graph).
+//
+// Launch sequence of sg_match for B pairs (P = M + N stacked rows per pair):
+//   encoder (1) -> n_stages x [QKV GEMM, attention, update-MLP layer 1 GEMM,
+//   update-MLP layer 2 GEMM + residual] -> final projection GEMM -> score GEMM
+//   -> persistent Sinkhorn with fused extraction.
+// The merge layer of the attention and the eval-mode BatchNorm are folded into
+// the first update-MLP layer at create time (all in float64 on the host):
+//   W1 [x || Wm m + bm] + b1, then BN  ==  W1' [x || m] + b1'
+//   with W1' = diag(s) [W1x | W1m Wm],  b1' = s (b1 + W1m bm - mean) + beta,
+//   s = gamma / sqrt(var + eps)
+// (update MLP of the realcat notes, "笔记：SuperGlue:Learning Feature Matching with
+// Graph Neural Networks论文阅读", section 多层GNN).
+#include "sg_internal.cuh"
+
+#include <cmath>
+#include <cstdlib>
+#include <cstring>
+#include <vector>
+
+using namespace sg;
+
+namespace {
+
+template <typename T> T* dmalloc(size_t n, bool* ok) {
+  void* p = nullptr;
+  if (n == 0) n = 1;
+  if (cudaMalloc(&p, n * sizeof(T)) != cudaSuccess) { *ok = false; return nullptr; }
+  return reinterpret_cast<T*>(p);
+}
+
+struct StageW {
+  void* Wqkv;        // 768 x 256 (bf16 or fp32)
+  float* bqkv;       // 768
+  void* W1;          // 512 x 512 folded
+  float* b1;         // 512 folded
+  void* W2;          // 256 x 512
+};
+
+struct GraphKey {
+  int B, M, N, kind;
+  const void* p[12];
+  bool operator==(const GraphKey& o) const { return std::memcmp(this, &o, sizeof(*this)) == 0; }
+};
+
+}  // namespace
+
+struct sg_handle {
+  sg_config cfg;
+  int device;
+  int num_sms;
+  bool bf16;
+  bool use_tc;
+  // weights
+  float* encW[SG_ENC_LAYERS];
+  float* encb[SG_ENC_LAYERS];
+  std::vector<StageW> stages;
+  void* Wf;
+  float* bf;
+  float alpha;
+  // workspace
+  float* x32;
+  __nv_bfloat16* x16;
+  void* qkv;
+  void* msg;
+  void* hid;
+  void* f;
+  float* Z;
+  unsigned char* sk_scratch;
+  size_t sk_scratch_bytes;
+  unsigned* status;
+  // host-buffer staging
+  float *s_k0, *s_c0, *s_d0, *s_k1, *s_c1, *s_d1, *s_logP, *s_ms0, *s_ms1;
+  int32_t *s_m0, *s_m1;
+  // graph cache
+  bool use_graph;
+  cudaStream_t cap_stream;
+  bool graph_valid;
+  GraphKey gkey;
+  cudaGraphExec_t gexec;
+  std::vector<void*> allocs;
+  sg_status_t sticky;
+};
+
+namespace {
+
+sg_status_t cuda_err(sg_handle* h, cudaError_t e) {
+  if (e == cudaSuccess) return SG_OK;
+  if (h) h->sticky = SG_ERR_CUDA;
+  return SG_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------- weight folding
+struct HostW {
+  std::vector<double> W;   // out x in
+  std::vector<double> b;
+  int out, in;
+};
+
+HostW load_linear(const float* W, const float* b, int out, int in) {
+  HostW r;
+  r.out = out; r.in = in;
+  r.W.assign(W, W + (size_t)out * in);
+  r.b.assign(out, 0.0);
+  if (b) for (int i = 0; i < out; ++i) r.b[i] = b[i];
+  return r;
+}
+
+void fold_bn(HostW& l, const float* const bn[4], double eps) {
+  for (int o = 0; o < l.out; ++o) {
+    const double s = (double)bn[0][o] / std::sqrt((double)bn[3][o] + eps);
+    for (int i = 0; i < l.in; ++i) l.W[(size_t)o * l.in + i] *= s;
+    l.b[o] = s * (l.b[o] - (double)bn[2][o]) + (double)bn[1][o];
+  }
+}
+
+template <typename T> T cvt(double v);
+template <> float cvt<float>(double v) { return (float)v; }
+template <> __nv_bfloat16 cvt<__nv_bfloat16>(double v) { return __float2bfloat16_rn((float)v); }
+
+template <typename T>
+void* upload_matrix(sg_handle* h, const std::vector<double>& W, size_t n, bool* ok) {
+  std::vector<T> tmp(n);
+  for (size_t i = 0; i < n; ++i) tmp[i] = cvt<T>(W[i]);
+  T* d = dmalloc<T>(n, ok);
+  if (!*ok) return nullptr;
+  h->allocs.push_back(d);
+  if (cudaMemcpy(d, tmp.data(), n * sizeof(T), cudaMemcpyHostToDevice) != cudaSuccess) *ok = false;
+  return d;
+}
+
+float* upload_f32(sg_handle* h, const std::vector<double>& v, bool* ok) {
+  return reinterpret_cast<float*>(upload_matrix<float>(h, v, v.size(), ok));
+}
+
+void* upload_w(sg_handle* h, const std::vector<double>& W, bool* ok) {
+  return h->bf16 ? upload_matrix<__nv_bfloat16>(h, W, W.size(), ok)
+                 : upload_matrix<float>(h, W, W.size(), ok);
+}
+
+sg_status_t pack_weights(sg_handle* h, const sg_weights* w) {
+  const sg_config& c = h->cfg;
+  const double eps = c.bn_eps;
+  bool ok = true;
+  static const int ch[6] = {3, 32, 64, 128, 256, 256};
+  for (int l = 0; l < SG_ENC_LAYERS; ++l) {
+    if (!w->enc_W[l]) return SG_ERR_INVALID_ARG;
+    if (l < SG_ENC_LAYERS - 1) {
+      if (!w->enc_b[l]) return SG_ERR_INVALID_ARG;
+      for (int k = 0; k < 4; ++k) if (!w->enc_bn[l][k]) return SG_ERR_INVALID_ARG;
+    }
+    HostW L = load_linear(w->enc_W[l], l < SG_ENC_LAYERS - 1 ? w->enc_b[l] : nullptr, ch[l + 1], ch[l]);
+    if (l < SG_ENC_LAYERS - 1) fold_bn(L, w->enc_bn[l], eps);
+    // transpose to in x out for the encoder kernel
+    std::vector<double> Wt((size_t)L.in * L.out);
+    for (int o = 0; o < L.out; ++o)
+      for (int i = 0; i < L.in; ++i) Wt[(size_t)i * L.out + o] = L.W[(size_t)o * L.in + i];
+    h->encW[l] = upload_f32(h, Wt, &ok);
+    h->encb[l] = upload_f32(h, L.b, &ok);
+  }
+  const int D = kD;
+  h->stages.resize(c.n_stages);
+  for (int s = 0; s < c.n_stages; ++s) {
+    if (!w->Wq[s] || !w->bq[s] || !w->Wk[s] || !w->bk[s] || !w->Wv[s] || !w->bv[s] ||
+        !w->Wm[s] || !w->bm[s] || !w->W1[s] || !w->b1[s] || !w->W2[s])
+      return SG_ERR_INVALID_ARG;
+    for (int k = 0; k < 4; ++k) if (!w->bn1[s][k]) return SG_ERR_INVALID_ARG;
+    std::vector<double> Wqkv((size_t)3 * D * D), bqkv(3 * D);
+    const float* Ws[3] = {w->Wq[s], w->Wk[s], w->Wv[s]};
+    const float* bs[3] = {w->bq[s], w->bk[s], w->bv[s]};
+    for (int t = 0; t < 3; ++t) {
+      for (size_t i = 0; i < (size_t)D * D; ++i) Wqkv[(size_t)t * D * D + i] = Ws[t][i];
+      for (int i = 0; i < D; ++i) bqkv[t * D + i] = bs[t][i];
+    }
+    // W1' = diag(s) [W1x | W1m Wm],  b1' = s (b1 + W1m bm - mean) + beta
+    const int D2 = 2 * D;
+    std::vector<double> W1f((size_t)D2 * D2), b1f(D2);
+    const float* W1 = w->W1[s];
+    const float* Wm = w->Wm[s];
+    const float* bm = w->bm[s];
+    std::vector<double> Wmd((size_t)D * D);
+    for (size_t i = 0; i < (size_t)D * D; ++i) Wmd[i] = Wm[i];
+    for (int o = 0; o < D2; ++o) {
+      const float* row = W1 + (size_t)o * D2;
+      for (int i = 0; i < D; ++i) W1f[(size_t)o * D2 + i] = row[i];
+      std::vector<double> acc(D, 0.0);
+      double bacc = w->b1[s][o];
+      for (int k = 0; k < D; ++k) {
+        const double wk = row[D + k];
+        const double* wm = &Wmd[(size_t)k * D];
+        for (int i = 0; i < D; ++i) acc[i] += wk * wm[i];
+        bacc += wk * bm[k];
+      }
+      for (int i = 0; i < D; ++i) W1f[(size_t)o * D2 + D + i] = acc[i];
+      b1f[o] = bacc;
+    }
+    HostW L1{W1f, b1f, D2, D2};
+    fold_bn(L1, w->bn1[s], eps);
+    std::vector<double> W2((size_t)D * D2);
+    for (size_t i = 0; i < (size_t)D * D2; ++i) W2[i] = w->W2[s][i];
+    StageW& st = h->stages[s];
+    st.Wqkv = upload_w(h, Wqkv, &ok);
+    st.bqkv = upload_f32(h, bqkv, &ok);
+    st.W1 = upload_w(h, L1.W, &ok);
+    st.b1 = upload_f32(h, L1.b, &ok);
+    st.W2 = upload_w(h, W2, &ok);
+  }
+  if (!w->Wf || !w->bf) return SG_ERR_INVALID_ARG;
+  std::vector<double> Wf(w->Wf, w->Wf + (size_t)D * D), bf(w->bf, w->bf + D);
+  h->Wf = upload_w(h, Wf, &ok);
+  h->bf = upload_f32(h, bf, &ok);
+  h->alpha = w->bin_score;
+  return ok ? SG_OK : SG_ERR_OOM;
+}
+
+// ---------------------------------------------------------------- launch sequence
+struct Inputs {
+  const float *k0, *c0, *d0, *k1, *c1, *d1;
+};
+
+cudaError_t gemm(sg_handle* h, const GemmArgs& g, int epi, bool out_bf16, int batch, cudaStream_t s,
+                 int* launches) {
+  ++*launches;
+  if (h->use_tc) return launch_gemm_tc(g, epi, batch, s);
+  return launch_gemm_simt(g, epi, h->bf16, out_bf16, batch, s);
+}
+
+// Steps 1-3: encoder, GNN, projection, scores -> S (B x M x lds, pair stride strideS)
+cudaError_t run_network(sg_handle* h, int B, int M, int N, const Inputs& in, float* S, long long lds,
+                        long long strideS, cudaStream_t s, int* launches) {
+  const sg_config& c = h->cfg;
+  const int P = M + N;
+  const int R = B * P;
+  const size_t esz = h->bf16 ? 2 : 4;
+  EncArgs ea{};
+  ea.kpts[0] = in.k0; ea.kpts[1] = in.k1;
+  ea.conf[0] = in.c0; ea.conf[1] = in.c1;
+  ea.desc[0] = in.d0; ea.desc[1] = in.d1;
+  for (int l = 0; l < SG_ENC_LAYERS; ++l) { ea.W[l] = h->encW[l]; ea.b[l] = h->encb[l]; }
+  ea.x32 = h->x32;
+  ea.x16 = h->x16;
+  ea.B = B; ea.M = M; ea.N = N;
+  ea.cx = c.img_w * 0.5f;
+  ea.cy = c.img_h * 0.5f;
+  const float mx = c.img_w > c.img_h ? c.img_w : c.img_h;
+  ea.inv_scale = (float)(1.0 / (c.norm_mode == 0 ? 0.7 * (double)mx : 0.5 * (double)mx));
+  cudaError_t e = launch_encoder(ea, h->bf16, s);
+  ++*launches;
+  if (e != cudaSuccess) return e;
+  const void* xin = h->bf16 ? (const void*)h->x16 : (const void*)h->x32;
+  for (int st = 0; st < c.n_stages; ++st) {
+    const StageW& w = h->stages[st];
+    GemmArgs g{};
+    // q|k|v = x Wqkv^T + b
+    g.A0 = xin; g.A1 = nullptr; g.lda = kD; g.k_split = kD;
+    g.W = w.Wqkv; g.bias = w.bqkv; g.out = h->qkv; g.ldo = kQKV;
+    g.rows = R; g.cols = kQKV; g.K = kD; g.scale = 1.f;
+    if ((e = gemm(h, g, EPI_BIAS, h->bf16, 1, s, launches)) != cudaSuccess) return e;
+    AttnArgs aa{};
+    aa.qkv = h->qkv; aa.msg = h->msg; aa.B = B; aa.M = M; aa.N = N;
+    aa.cross = (st % 2 == 1);
+    aa.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)kDh));
+    ++*launches;
+    e = h->use_tc ? launch_attention_tc(aa, s) : launch_attention_simt(aa, h->bf16, s);
+    if (e != cudaSuccess) return e;
+    // h = relu(W1' [x || m] + b1')
+    g = GemmArgs{};
+    g.A0 = xin; g.A1 = h->msg; g.lda = kD; g.k_split = kD;
+    g.W = w.W1; g.bias = w.b1; g.out = h->hid; g.ldo = 2 * kD;
+    g.rows = R; g.cols = 2 * kD; g.K = 2 * kD; g.scale = 1.f;
+    if ((e = gemm(h, g, EPI_BIAS_RELU, h->bf16, 1, s, launches)) != cudaSuccess) return e;
+    // x += W2 h   (bias 0), refresh the bf16 shadow
+    g = GemmArgs{};
+    g.A0 = h->hid; g.A1 = nullptr; g.lda = 2 * kD; g.k_split = 2 * kD;
+    g.W = w.W2; g.bias = nullptr; g.out = h->x32; g.out2 = h->x16; g.ldo = kD;
+    g.rows = R; g.cols = kD; g.K = 2 * kD; g.scale = 1.f;
+    if ((e = gemm(h, g, EPI_RESIDUAL, h->bf16, 1, s, launches)) != cudaSuccess) return e;
+  }
+  // f = Wf x + bf
+  GemmArgs g{};
+  g.A0 = xin; g.A1 = nullptr; g.lda = kD; g.k_split = kD;
+  g.W = h->Wf; g.bias = h->bf; g.out = h->f; g.ldo = kD;
+  g.rows = R; g.cols = kD; g.K = kD; g.scale = 1.f;
+  if ((e = gemm(h, g, EPI_BIAS, h->bf16, 1, s, launches)) != cudaSuccess) return e;
+  // S_b = f_A f_B^T / sqrt(D), batched over pairs
+  g = GemmArgs{};
+  g.A0 = h->f; g.A1 = nullptr; g.lda = kD; g.k_split = kD;
+  g.W = (const unsigned char*)h->f + (size_t)M * kD * esz;
+  g.out = S; g.ldo = lds;
+  g.rows = M; g.cols = N; g.K = kD;
+  g.strideA = (long long)P * kD; g.strideW = (long long)P * kD; g.strideO = strideS;
+  g.scale = (float)(1.0 / std::sqrt((double)kD));
+  return gemm(h, g, EPI_SCALE, false, B, s, launches);
+}
+
+// Steps 4-5 from S.
+cudaError_t run_transport(sg_handle* h, int B, int M, int N, const float* S, long long lds,
+                          long long strideS, float* logP, int32_t* m0, int32_t* m1, float* s0,
+                          float* s1, cudaStream_t st, int* launches) {
+  const size_t C = N + 1, R = M + 1;
+  unsigned char* p = h->sk_scratch;
+  SinkhornArgs a{};
+  a.barrier = reinterpret_cast<unsigned*>(p);
+  a.abort_flag = a.barrier + B;
+  size_t off = ((B + 1) * sizeof(unsigned) + 255) & ~(size_t)255;
+  a.acc = reinterpret_cast<float*>(p + off);
+  a.fb = a.acc + (size_t)B * 3 * C;
+  off += (size_t)B * 5 * C * 4;
+  off = (off + 255) & ~(size_t)255;
+  a.colbest = reinterpret_cast<unsigned long long*>(p + off);
+  off += (size_t)B * N * 8;
+  off = (off + 255) & ~(size_t)255;
+  const size_t zero_bytes = off;
+  a.u = reinterpret_cast<float*>(p + off);
+  off += (size_t)B * R * 4;
+  off = (off + 255) & ~(size_t)255;
+  a.idx0 = reinterpret_cast<int32_t*>(p + off);
+  off += (size_t)B * M * 4;
+  off = (off + 255) & ~(size_t)255;
+  a.max0 = reinterpret_cast<float*>(p + off);
+  cudaError_t e = cudaMemsetAsync(p, 0, zero_bytes, st);
+  if (e != cudaSuccess) return e;
+  a.S = S; a.lds = lds; a.strideS = strideS; a.alpha = h->alpha;
+  a.B = B; a.M = M; a.N = N; a.iters = h->cfg.sinkhorn_iters;
+  a.threshold = h->cfg.match_threshold;
+  a.logP = logP; a.matches0 = m0; a.matches1 = m1; a.mscores0 = s0; a.mscores1 = s1;
+  a.status = h->status;
+  a.timeout_ns = 1000000000ull;   // 1 s per barrier wait
+  return launch_sinkhorn(a, h->num_sms, st, launches);
+}
+
+sg_status_t check_shape(sg_handle* h, int B, int M, int N) {
+  if (!h) return SG_ERR_INVALID_ARG;
+  if (B < 0 || M < 0 || N < 0) return SG_ERR_SHAPE;
+  if (B > h->cfg.max_B || M > h->cfg.max_M || N > h->cfg.max_N) return SG_ERR_SHAPE;
+  return SG_OK;
+}
+
+sg_status_t empty_outputs(sg_handle* h, int B, int M, int N, int32_t* m0, int32_t* m1, float* s0,
+                          float* s1, cudaStream_t s) {
+  cudaError_t e = cudaSuccess;
+  if (B * M > 0) {
+    if (!m0 || !s0) return SG_ERR_INVALID_ARG;
+    e = cudaMemsetAsync(m0, 0xff, (size_t)B * M * sizeof(int32_t), s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(s0, 0, (size_t)B * M * sizeof(float), s);
+  }
+  if (e == cudaSuccess && B * N > 0) {
+    if (!m1 || !s1) return SG_ERR_INVALID_ARG;
+    e = cudaMemsetAsync(m1, 0xff, (size_t)B * N * sizeof(int32_t), s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(s1, 0, (size_t)B * N * sizeof(float), s);
+  }
+  return cuda_err(h, e);
+}
+
+// Run `fn` (which enqueues work on a stream) either directly or through a
+// cached CUDA graph keyed by the call's sizes and pointers.
+template <typename F>
+sg_status_t run_maybe_graph(sg_handle* h, const GraphKey& key, cudaStream_t s, F&& fn) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (s) cudaStreamIsCapturing(s, &cs);
+  if (!h->use_graph || cs != cudaStreamCaptureStatusNone) {
+    int launches = 0;
+    return cuda_err(h, fn(s, &launches));
+  }
+  if (!(h->graph_valid && h->gkey == key)) {
+    cudaGraph_t g = nullptr;
+    cudaError_t e = cudaStreamBeginCapture(h->cap_stream, cudaStreamCaptureModeThreadLocal);
+    if (e != cudaSuccess) return cuda_err(h, e);
+    int launches = 0;
+    cudaError_t fe = fn(h->cap_stream, &launches);
+    e = cudaStreamEndCapture(h->cap_stream, &g);
+    if (fe != cudaSuccess || e != cudaSuccess) {
+      if (g) cudaGraphDestroy(g);
+      cudaGetLastError();
+      return cuda_err(h, fe != cudaSuccess ? fe : e);
+    }
+    bool updated = false;
+    if (h->graph_valid) {
+      cudaGraphExecUpdateResultInfo info;
+      if (cudaGraphExecUpdate(h->gexec, g, &info) == cudaSuccess) updated = true;
+      else cudaGetLastError();
+    }
+    if (!updated) {
+      if (h->graph_valid) cudaGraphExecDestroy(h->gexec);
+      h->graph_valid = false;
+      e = cudaGraphInstantiate(&h->gexec, g, 0);
+      if (e != cudaSuccess) { cudaGraphDestroy(g); return cuda_err(h, e); }
+    }
+    cudaGraphDestroy(g);
+    h->graph_valid = true;
+    h->gkey = key;
+  }
+  return cuda_err(h, cudaGraphLaunch(h->gexec, s));
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* sg_strerror(sg_status_t s) {
+  switch (s) {
+    case SG_OK: return "ok";
+    case SG_ERR_INVALID_ARG: return "invalid argument";
+    case SG_ERR_SHAPE: return "size outside the handle's configured maxima";
+    case SG_ERR_OOM: return "device allocation failed";
+    case SG_ERR_CUDA: return "CUDA runtime error";
+    case SG_ERR_TIMEOUT: return "a bounded device-side wait ran out";
+    case SG_ERR_NUMERIC: return "non-finite value in the transport solver";
+    case SG_ERR_UNSUPPORTED: return "unsupported device or configuration";
+  }
+  return "unknown status";
+}
+
+int sg_launches_per_match(const sg_handle* h, int B, int M, int N) {
+  if (!h || B == 0 || M == 0 || N == 0) return 0;
+  return 4 + 4 * h->cfg.n_stages;
+}
+
+sg_status_t sg_create(const sg_weights* w, const sg_config* cfg, sg_handle** out) {
+  if (!out) return SG_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (!w || !cfg) return SG_ERR_INVALID_ARG;
+  if (cfg->D != kD || cfg->H != kH) return SG_ERR_UNSUPPORTED;
+  if (cfg->n_stages < 1 || cfg->n_stages > SG_MAX_STAGES || cfg->sinkhorn_iters < 0 ||
+      cfg->max_B < 0 || cfg->max_M < 0 || cfg->max_N < 0 || !(cfg->bn_eps >= 0.f) ||
+      !(cfg->img_w > 0.f) || !(cfg->img_h > 0.f) || (cfg->norm_mode != 0 && cfg->norm_mode != 1) ||
+      (cfg->precision != SG_PRECISION_FP32 && cfg->precision != SG_PRECISION_BF16))
+    return SG_ERR_INVALID_ARG;
+  if (cfg->max_N + 1 > 16384) return SG_ERR_UNSUPPORTED;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return SG_ERR_UNSUPPORTED; }
+  cudaDeviceProp prop;
+  if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return SG_ERR_CUDA;
+  if (prop.major != 10) return SG_ERR_UNSUPPORTED;
+
+  sg_handle* h = new sg_handle();
+  h->cfg = *cfg;
+  h->device = dev;
+  h->num_sms = prop.multiProcessorCount;
+  h->bf16 = cfg->precision == SG_PRECISION_BF16;
+  h->use_tc = h->bf16 && tc_available() && std::getenv("SG_FORCE_SIMT") == nullptr;
+  h->use_graph = std::getenv("SG_NO_GRAPH") == nullptr;
+  h->sticky = SG_OK;
+  sg_status_t st = pack_weights(h, w);
+  if (st != SG_OK) { sg_destroy(h); return st; }
+  bool ok = true;
+  const size_t Bm = cfg->max_B, Mm = cfg->max_M, Nm = cfg->max_N;
+  const size_t R = Bm * (Mm + Nm);
+  const size_t esz = h->bf16 ? 2 : 4;
+  auto al = [&](size_t bytes) -> void* {
+    void* p = dmalloc<unsigned char>(bytes + 256, &ok);
+    if (p) h->allocs.push_back(p);
+    return p;
+  };
+  h->x32 = (float*)al(R * kD * 4);
+  h->x16 = h->bf16 ? (__nv_bfloat16*)al(R * kD * 2) : nullptr;
+  h->qkv = al(R * kQKV * esz);
+  h->msg = al(R * kD * esz);
+  h->hid = al(R * 2 * kD * esz);
+  h->f = al(R * kD * esz);
+  h->Z = (float*)al(Bm * Mm * ((Nm + 3) & ~(size_t)3) * 4);
+  h->sk_scratch_bytes = sinkhorn_scratch_bytes((int)Bm, (int)Mm, (int)Nm);
+  h->sk_scratch = (unsigned char*)al(h->sk_scratch_bytes);
+  h->status = (unsigned*)al(sizeof(unsigned));
+  h->s_k0 = (float*)al(Bm * Mm * 2 * 4);
+  h->s_c0 = (float*)al(Bm * Mm * 4);
+  h->s_d0 = (float*)al(Bm * Mm * kD * 4);
+  h->s_k1 = (float*)al(Bm * Nm * 2 * 4);
+  h->s_c1 = (float*)al(Bm * Nm * 4);
+  h->s_d1 = (float*)al(Bm * Nm * kD * 4);
+  h->s_logP = (float*)al(Bm * (Mm + 1) * (Nm + 1) * 4);
+  h->s_m0 = (int32_t*)al(Bm * Mm * 4);
+  h->s_m1 = (int32_t*)al(Bm * Nm * 4);
+  h->s_ms0 = (float*)al(Bm * Mm * 4);
+  h->s_ms1 = (float*)al(Bm * Nm * 4);
+  if (!ok) { cudaGetLastError(); sg_destroy(h); return SG_ERR_OOM; }
+  if (cudaMemset(h->status, 0, sizeof(unsigned)) != cudaSuccess ||
+      cudaStreamCreateWithFlags(&h->cap_stream, cudaStreamNonBlocking) != cudaSuccess) {
+    sg_destroy(h);
+    return SG_ERR_CUDA;
+  }
+  *out = h;
+  return SG_OK;
+}
+
+void sg_destroy(sg_handle* h) {
+  if (!h) return;
+  cudaDeviceSynchronize();
+  if (h->graph_valid) cudaGraphExecDestroy(h->gexec);
+  if (h->cap_stream) cudaStreamDestroy(h->cap_stream);
+  for (void* p : h->allocs) cudaFree(p);
+  delete h;
+}
+
+sg_status_t sg_scores(sg_handle* h, int B, int M, int N, const float* kpts0, const float* conf0,
+                      const float* desc0, const float* kpts1, const float* conf1, const float* desc1,
+                      float* out_scores, void* stream) {
+  sg_status_t st = check_shape(h, B, M, N);
+  if (st != SG_OK) return st;
+  if (B == 0) return SG_OK;
+  if (M == 0 || N == 0) return SG_ERR_SHAPE;
+  if (!kpts0 || !conf0 || !desc0 || !kpts1 || !conf1 || !desc1 || !out_scores)
+    return SG_ERR_INVALID_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  Inputs in{kpts0, conf0, desc0, kpts1, conf1, desc1};
+  int launches = 0;
+  return cuda_err(h, run_network(h, B, M, N, in, out_scores, N, (long long)M * N, s, &launches));
+}
+
+sg_status_t sg_optimal_transport(sg_handle* h, int B, int M, int N, const float* scores,
+                                 float* out_logP, int32_t* matches0, int32_t* matches1,
+                                 float* mscores0, float* mscores1, void* stream) {
+  sg_status_t st = check_shape(h, B, M, N);
+  if (st != SG_OK) return st;
+  if (B == 0) return SG_OK;
+  if (M == 0 || N == 0) return SG_ERR_SHAPE;
+  if (!scores || !matches0 || !matches1 || !mscores0 || !mscores1) return SG_ERR_INVALID_ARG;
+  int launches = 0;
+  return cuda_err(h, run_transport(h, B, M, N, scores, N, (long long)M * N, out_logP, matches0,
+                                   matches1, mscores0, mscores1, (cudaStream_t)stream, &launches));
+}
+
+sg_status_t sg_match(sg_handle* h, int B, int M, int N, const float* kpts0, const float* conf0,
+                     const float* desc0, const float* kpts1, const float* conf1, const float* desc1,
+                     float* out_logP, int32_t* matches0, int32_t* matches1, float* mscores0,
+                     float* mscores1, void* stream) {
+  sg_status_t st = check_shape(h, B, M, N);
+  if (st != SG_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (B == 0) return SG_OK;
+  if (M == 0 || N == 0) return empty_outputs(h, B, M, N, matches0, matches1, mscores0, mscores1, s);
+  if (!kpts0 || !conf0 || !desc0 || !kpts1 || !conf1 || !desc1 || !matches0 || !matches1 ||
+      !mscores0 || !mscores1)
+    return SG_ERR_INVALID_ARG;
+  const long long lds = (N + 3) & ~3;
+  const long long strideS = (long long)M * lds;
+  Inputs in{kpts0, conf0, desc0, kpts1, conf1, desc1};
+  GraphKey key{};
+  key.B = B; key.M = M; key.N = N; key.kind = 1;
+  const void* ps[12] = {kpts0, conf0, desc0, kpts1, conf1, desc1, out_logP, matches0, matches1,
+                        mscores0, mscores1, nullptr};
+  std::memcpy(key.p, ps, sizeof(ps));
+  return run_maybe_graph(h, key, s, [&](cudaStream_t cs, int* launches) -> cudaError_t {
+    cudaError_t e = run_network(h, B, M, N, in, h->Z, lds, strideS, cs, launches);
+    if (e != cudaSuccess) return e;
+    return run_transport(h, B, M, N, h->Z, lds, strideS, out_logP, matches0, matches1, mscores0,
+                         mscores1, cs, launches);
+  });
+}
+
+sg_status_t sg_match_host(sg_handle* h, int B, int M, int N, const float* kpts0, const float* conf0,
+                          const float* desc0, const float* kpts1, const float* conf1,
+                          const float* desc1, float* out_logP, int32_t* matches0, int32_t* matches1,
+                          float* mscores0, float* mscores1, void* stream) {
+  sg_status_t st = check_shape(h, B, M, N);
+  if (st != SG_OK) return st;
+  if (B == 0) return SG_OK;
+  cudaStream_t s = (cudaStream_t)stream;
+  const size_t nM = (size_t)B * M, nN = (size_t)B * N;
+  auto h2d = [&](void* d, const void* src, size_t bytes) -> cudaError_t {
+    if (bytes == 0) return cudaSuccess;
+    return cudaMemcpyAsync(d, src, bytes, cudaMemcpyHostToDevice, s);
+  };
+  auto d2h = [&](void* dst, const void* d, size_t bytes) -> cudaError_t {
+    if (bytes == 0) return cudaSuccess;
+    return cudaMemcpyAsync(dst, d, bytes, cudaMemcpyDeviceToHost, s);
+  };
+  if ((nM && (!matches0 || !mscores0)) || (nN && (!matches1 || !mscores1))) return SG_ERR_INVALID_ARG;
+  if (M > 0 && N > 0) {
+    if (!kpts0 || !conf0 || !desc0 || !kpts1 || !conf1 || !desc1) return SG_ERR_INVALID_ARG;
+    cudaError_t e = h2d(h->s_k0, kpts0, nM * 8);
+    if (e == cudaSuccess) e = h2d(h->s_c0, conf0, nM * 4);
+    if (e == cudaSuccess) e = h2d(h->s_d0, desc0, nM * kD * 4);
+    if (e == cudaSuccess) e = h2d(h->s_k1, kpts1, nN * 8);
+    if (e == cudaSuccess) e = h2d(h->s_c1, conf1, nN * 4);
+    if (e == cudaSuccess) e = h2d(h->s_d1, desc1, nN * kD * 4);
+    if (e != cudaSuccess) return cuda_err(h, e);
+  }
+  st = sg_match(h, B, M, N, h->s_k0, h->s_c0, h->s_d0, h->s_k1, h->s_c1, h->s_d1,
+                out_logP ? h->s_logP : nullptr, h->s_m0, h->s_m1, h->s_ms0, h->s_ms1, stream);
+  if (st != SG_OK) return st;
+  cudaError_t e = d2h(matches0, h->s_m0, nM * 4);
+  if (e == cudaSuccess) e = d2h(matches1, h->s_m1, nN * 4);
+  if (e == cudaSuccess) e = d2h(mscores0, h->s_ms0, nM * 4);
+  if (e == cudaSuccess) e = d2h(mscores1, h->s_ms1, nN * 4);
+  if (e == cudaSuccess && out_logP && M > 0 && N > 0)
+    e = d2h(out_logP, h->s_logP, (size_t)B * (M + 1) * (N + 1) * 4);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  return cuda_err(h, e);
+}
+
+sg_status_t sg_selftest_barrier_timeout(sg_handle* h, unsigned timeout_us, void* stream) {
+  if (!h) return SG_ERR_INVALID_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  unsigned* scratch = reinterpret_cast<unsigned*>(h->sk_scratch);
+  int* returned = reinterpret_cast<int*>(h->sk_scratch + 16);
+  cudaError_t e = cudaMemsetAsync(h->sk_scratch, 0, 32, s);
+  if (e == cudaSuccess)
+    e = launch_barrier_selftest(scratch, h->status, (unsigned long long)timeout_us * 1000ull, returned, s);
+  int ret = 0;
+  if (e == cudaSuccess) e = cudaMemcpyAsync(&ret, returned, sizeof(int), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_err(h, e);
+  if (ret != 1) return SG_ERR_INVALID_ARG;   // the wait did not report its expiry
+  return sg_status(h, stream);
+}
+
+sg_status_t sg_status(sg_handle* h, void* stream) {
+  if (!h) return SG_ERR_INVALID_ARG;
+  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_err(h, e);
+  unsigned word = 0;
+  e = cudaMemcpy(&word, h->status, sizeof(unsigned), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_err(h, e);
+  if (word) cudaMemset(h->status, 0, sizeof(unsigned));
+  sg_status_t sticky = h->sticky;
+  h->sticky = SG_OK;
+  if (sticky != SG_OK) return sticky;
+  if (word & kStatusTimeout) return SG_ERR_TIMEOUT;
+  if (word & kStatusNumeric) return SG_ERR_NUMERIC;
+  return SG_OK;
+}
+
+}  // extern "C"

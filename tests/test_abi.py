@@ -1,0 +1,62 @@
+"""The C-ABI library builds, loads and exports every entry point include/sg.h
+declares; host-side argument checks (no GPU compute)."""
+import ctypes as C
+import os
+import re
+import subprocess
+
+import pytest
+
+from conftest import ROOT
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from learned_sparse_feature_b200 import build, binding
+    build.build()
+    return binding.load()
+
+
+def _declared():
+    text = open(os.path.join(ROOT, "include", "sg.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(sg_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for n in ("sg_create", "sg_match", "sg_destroy", "sg_status"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    from learned_sparse_feature_b200 import binding
+    out = subprocess.run(["nm", "-D", "--defined-only", binding.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r" T (sg_\w+)", out))
+    for n in _declared():
+        assert n in exported, n
+        assert hasattr(lib, n)
+    assert set(binding.EXPORTED) == set(_declared())
+
+
+def test_strerror_and_null_handle(lib):
+    assert lib.sg_strerror(0) == b"ok"
+    assert lib.sg_strerror(5).startswith(b"a bounded")
+    # null handle -> INVALID_ARG, synchronously, no device work
+    assert lib.sg_match(None, 1, 1, 1, *([None] * 12)) == 1
+    assert lib.sg_status(None, None) == 1
+    assert lib.sg_launches_per_match(None, 1, 1, 1) == 0
+
+
+def test_create_rejects_bad_arguments(lib):
+    from learned_sparse_feature_b200 import binding
+    h = C.c_void_p()
+    assert lib.sg_create(None, None, C.byref(h)) == 1
+    w = binding.SgWeights()
+    cfg = binding.SgConfig(128, 4, 18, 100, 0.2, 1e-5, 1, 640.0, 480.0, 0, 1, 64, 64)
+    assert lib.sg_create(C.byref(w), C.byref(cfg), C.byref(h)) == 7     # D != 256
+    cfg = binding.SgConfig(256, 4, 0, 100, 0.2, 1e-5, 1, 640.0, 480.0, 0, 1, 64, 64)
+    assert lib.sg_create(C.byref(w), C.byref(cfg), C.byref(h)) == 1     # n_stages = 0
+    cfg = binding.SgConfig(256, 4, 18, 100, 0.2, 1e-5, 5, 640.0, 480.0, 0, 1, 64, 64)
+    assert lib.sg_create(C.byref(w), C.byref(cfg), C.byref(h)) == 1     # bad precision
+    assert not h.value
