@@ -1,0 +1,404 @@
+"""Benchmark of the SuperGlue matcher forward pass on B200 through libsg.
+
+One step = the whole hot path (encoder, 18 attentional stages, projection,
+score matrix, 100 Sinkhorn iterations, extraction) on one batch of synthetic
+pairs whose inputs are already resident in HBM.  Default workload: one pair of
+M = N = 2048 keypoints, bf16 operands.  Prints one JSON line (rank 0).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+Multi-GPU: pairs are independent, so every rank matches its own pairs with no
+collective on the data path (weak scaling); the step time is the max over
+ranks.  ``--impl reference`` times the float64 CPU oracle (test infrastructure)
+on the same workload, on a bounded sample per step.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from learned_sparse_feature_b200 import synth  # noqa: E402
+
+METRIC = "matched pairs/sec & ms/pair at M=N=2048 (L=9,T=100); % of roofline"
+UNIT = "pairs/s"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# --------------------------------------------------------------------------- host logic
+def shard_pairs(pairs_per_rank: int, rank: int):
+    """First pair index of a rank: rank r matches pairs [r*B, (r+1)*B) of the workload's stream."""
+    return rank * pairs_per_rank
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in FALLBACK_PEAKS}, "measured"
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def algorithmic_work(B, M, N, n_stages=18, T=100, D=256):
+    """Per-launch algorithmic work of each kernel class (FLOPs, or bytes for Sinkhorn)."""
+    P = M + N
+    R = B * P
+    self_pairs = B * (M * M + N * N)
+    cross_pairs = B * 2 * M * N
+    n_self = (n_stages + 1) // 2
+    n_cross = n_stages // 2
+    attn_flops = 4 * D * (n_self * self_pairs + n_cross * cross_pairs) / n_stages
+    E = (M + 1) * (N + 1)
+    return {
+        "encoder": ("alu", 2.0 * R * (3 * 32 + 32 * 64 + 64 * 128 + 128 * 256 + 256 * 256)),
+        "qkv_gemm": ("tensor", 2.0 * R * 3 * D * D),
+        "attention": ("tensor", float(attn_flops)),
+        "mlp1_gemm": ("tensor", 2.0 * R * (2 * D) * (2 * D)),
+        "mlp2_gemm": ("tensor", 2.0 * R * D * (2 * D)),
+        "proj_gemm": ("tensor", 2.0 * R * D * D),
+        "score_gemm": ("tensor", 2.0 * B * M * N * D),
+        # the spec model of Sinkhorn traffic: 2 passes over E fp32 per iteration
+        "sinkhorn": ("hbm", 2.0 * T * 4 * E * B),
+    }
+
+
+class ClockSampler:
+    """nvidia-smi SM clock / throttle-reason sampling during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"sg_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx = float(parts[2])
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------- oracle sample
+def oracle_step(batch, weights, pair=0, stages_sampled=2, iters_sampled=10):
+    """Time the float64 oracle on a bounded sample of one pair and extrapolate
+    to the whole pair: encoder, `stages_sampled` attentional stages (one self,
+    one cross) of the 18, projection + scores, `iters_sampled` of the 100
+    Sinkhorn iterations, extraction.  Returns (seconds per pair, description)."""
+    from oracle import superglue_oracle as O
+    k0, c0, d0 = batch["kpts0"][pair], batch["conf0"][pair], batch["desc0"][pair]
+    k1, c1, d1 = batch["kpts1"][pair], batch["conf1"][pair], batch["desc1"][pair]
+    t0 = time.perf_counter()
+    x0 = O.keypoint_encoder(O.normalize_keypoints(k0, synth.IMG_W, synth.IMG_H), c0, d0, weights, synth.BN_EPS)
+    x1 = O.keypoint_encoder(O.normalize_keypoints(k1, synth.IMG_W, synth.IMG_H), c1, d1, weights, synth.BN_EPS)
+    t1 = time.perf_counter()
+    x0, x1 = O.attentional_gnn(x0, x1, weights, synth.H, synth.BN_EPS, n_stages=stages_sampled)
+    t2 = time.perf_counter()
+    S = O.score_matrix(x0, x1, weights["Wf"], weights["bf"])
+    t3 = time.perf_counter()
+    logP = O.log_optimal_transport(S, float(weights["bin_score"]), iters_sampled)
+    t4 = time.perf_counter()
+    O.extract_matches(logP, synth.MATCH_THRESHOLD)
+    t5 = time.perf_counter()
+    per_pair = ((t1 - t0) + (t2 - t1) * (synth.N_STAGES / stages_sampled) + (t3 - t2)
+                + (t4 - t3) * (synth.SINKHORN_ITERS / iters_sampled) + (t5 - t4))
+    desc = (f"1 pair of {len(k0)}x{len(k1)}: encoder, {stages_sampled} of {synth.N_STAGES} stages, "
+            f"scores, {iters_sampled} of {synth.SINKHORN_ITERS} Sinkhorn iterations, extraction; "
+            f"scaled to the whole pair ({t5 - t0:.1f} s measured)")
+    return per_pair, desc
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+# --------------------------------------------------------------------------- arms
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return None
+    weights = synth.make_weights(0)
+    batch = synth.make_batch(w, 0, 1)
+    for _ in range(args.warmup):
+        oracle_step(batch, weights)
+    times = []
+    desc = ""
+    for _ in range(args.steps):
+        t, desc = oracle_step(batch, weights)
+        times.append(t)
+    ms = 1000.0 * float(np.mean(times))
+    value = 1000.0 / ms
+    cores = cpu_cores()
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "ms_per_pair": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": _config(w, args.gpus),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def _config(w, n_gpus):
+    return {"workload": w.name, "B_per_gpu": w.B, "M": w.M, "N": w.N, "stages": synth.N_STAGES,
+            "sinkhorn_iters": synth.SINKHORN_ITERS, "precision": w.precision,
+            "parallelism": f"replicas{n_gpus}", "l2": "flushed (256 MiB write) before every timed step"}
+
+
+def run_native(args, w):
+    import torch
+    import torch.distributed as dist
+
+    from learned_sparse_feature_b200 import build
+    from learned_sparse_feature_b200.binding import Matcher
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if rank == 0:
+        build.build()
+    if world > 1:
+        dist.barrier()
+    B, M, N = w.B, w.M, w.N
+
+    # CPU baseline first (rank 0, N=1 only), before the GPU work starts
+    cpu_baseline = None
+    weights = synth.make_weights(0)
+    batch = synth.make_batch(w, shard_pairs(B, rank), B)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        t, desc = oracle_step(batch, weights)
+        cpu_baseline = {"value": 1.0 / t, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle", "sample": desc}
+
+    m = Matcher(weights, B, M, N, precision=w.precision)
+    t = {k: torch.from_numpy(np.ascontiguousarray(batch[k])).to(dev)
+         for k in ("kpts0", "conf0", "desc0", "kpts1", "conf1", "desc1")}
+    logP = torch.empty((B, M + 1, N + 1), dtype=torch.float32, device=dev)
+    m0 = torch.empty((B, M), dtype=torch.int32, device=dev)
+    m1 = torch.empty((B, N), dtype=torch.int32, device=dev)
+    s0 = torch.empty((B, M), dtype=torch.float32, device=dev)
+    s1 = torch.empty((B, N), dtype=torch.float32, device=dev)
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        m.match(t["kpts0"], t["conf0"], t["desc0"], t["kpts1"], t["conf1"], t["desc1"],
+                logP, m0, m1, s0, s1, stream)
+
+    def timed(fn, K, profile=False):
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+        per_class = {}
+        total = 0.0
+        for i in range(K):
+            flush.zero_()
+            evs[i][0].record(stream)
+            fn()
+            evs[i][1].record(stream)
+            if profile:
+                torch.cuda.synchronize()
+                for k, (ms, n) in m.profile_read().items():
+                    a = per_class.setdefault(k, [0.0, 0])
+                    a[0] += ms
+                    a[1] += n
+        torch.cuda.synchronize()
+        for s, e in evs:
+            total += s.elapsed_time(e)
+        return total, per_class
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st = m.status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} after warm-up")
+
+    clocks = ClockSampler(torch.cuda.current_device())
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    total_ms, _ = timed(step, args.steps)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if world > 1:
+        dist.barrier()
+    tt = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+    total_ms = float(tt.item())
+    ms_per_step = total_ms / args.steps
+    pairs = B * world * args.steps
+    value = pairs / (total_ms / 1000.0)
+
+    # per-kernel breakdown: same steps with events between the launches
+    m.profile(True)
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize()
+    _, per_class = timed(step, args.steps, profile=True)
+    m.profile(False)
+    st = m.status()
+    if st != 0:
+        raise RuntimeError(f"device status {st}")
+
+    # end to end through the host-buffer entry point (pinned memory, copies timed)
+    host = {k: torch.from_numpy(np.ascontiguousarray(batch[k])).pin_memory()
+            for k in ("kpts0", "conf0", "desc0", "kpts1", "conf1", "desc1")}
+    hm0 = torch.empty((B, M), dtype=torch.int32).pin_memory()
+    hm1 = torch.empty((B, N), dtype=torch.int32).pin_memory()
+    hs0 = torch.empty((B, M), dtype=torch.float32).pin_memory()
+    hs1 = torch.empty((B, N), dtype=torch.float32).pin_memory()
+
+    def e2e_step():
+        m.match_host(host["kpts0"], host["conf0"], host["desc0"], host["kpts1"], host["conf1"],
+                     host["desc1"], None, hm0, hm1, hs0, hs1, stream)
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    e2e_ms, _ = timed(e2e_step, args.steps)
+    te = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_ms = float(te.item())
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = sum(v.numel() * v.element_size() for v in (hm0, hm1, hs0, hs1))
+
+    # roofline of the dominant kernel class
+    peaks, peak_src = load_peaks()
+    work = algorithmic_work(B, M, N)
+    dom = max(per_class, key=lambda k: per_class[k][0])
+    ms_dom, n_dom = per_class[dom]
+    bound, units = work[dom]
+    avg_s = ms_dom / n_dom / 1000.0
+    if bound == "hbm":
+        achieved, peak, unit = units / avg_s / 1e9, peaks["hbm_gbs"], "GB/s"
+    elif bound == "tensor":
+        achieved, peak, unit = units / avg_s / 1e12, peaks["bf16_tflops"], "TFLOP/s"
+    else:
+        achieved, peak, unit = units / avg_s / 1e12, None, "TFLOP/s"
+    roofline = {"bound": bound, "kernel": dom, "achieved": achieved, "peak": peak, "unit": unit,
+                "frac": (achieved / peak) if peak else None, "traffic": None,
+                "peak_source": peak_src + (" (burst)" if bound == "tensor" else "")}
+    breakdown = {}
+    for k, (ms, n) in per_class.items():
+        if n == 0:
+            continue
+        b, u = work[k]
+        avg = ms / n / 1000.0
+        if b == "hbm":
+            rate = {"GB/s": u / avg / 1e9, "frac_hbm": u / avg / 1e9 / peaks["hbm_gbs"]}
+        else:
+            r = u / avg / 1e12
+            rate = {"TFLOP/s": r}
+            if b == "tensor":
+                rate["frac_tensor"] = r / peaks["bf16_tflops"]
+        breakdown[k] = {"ms_per_step": ms / args.steps, "launches_per_step": n // args.steps, **rate}
+    gnn = [k for k in ("qkv_gemm", "attention", "mlp1_gemm", "mlp2_gemm", "proj_gemm", "score_gemm")
+           if k in per_class]
+    gnn_flops = sum(work[k][1] * per_class[k][1] for k in gnn)
+    gnn_s = sum(per_class[k][0] for k in gnn) / 1000.0
+
+    out = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "ms_per_pair": ms_per_step / B,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if w.precision == "bf16" else "f32",
+        "data": "synthetic (seeded keypoint pairs, random-init weights)",
+        "config": _config(w, world),
+        "roofline": roofline,
+        "gnn_tensor_frac": (gnn_flops / gnn_s / 1e12 / peaks["bf16_tflops"]) if gnn_s > 0 else None,
+        "kernels": breakdown,
+        "e2e": {"value": B * world * args.steps / (e2e_ms / 1000.0), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "note": "sg_match_host: pinned H2D of inputs, pass, D2H of matches and scores"},
+        "gpu_launches": m.launches_per_match(B, M, N) * args.steps,
+        "clocks": clk,
+        "cpu_baseline": cpu_baseline,
+    }
+    m.close()
+    return out if rank == 0 else None
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="pair2048", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    w = synth.WORKLOADS[args.workload]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if args.impl == "reference":
+        res = run_reference(args, w)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        res = run_native(args, w)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    if res is not None:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

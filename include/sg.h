@@ -207,6 +207,19 @@ sg_status_t sg_status(sg_handle* h, void* stream);
  */
 sg_status_t sg_selftest_barrier_timeout(sg_handle* h, unsigned timeout_us, void* stream);
 
+/*
+ * Per-kernel timing.  While enabled, sg_match records a CUDA event before every
+ * kernel (and the Sinkhorn scratch clear) and one after the last; the events
+ * are part of the captured graph.  After the stream has been synchronised,
+ * sg_profile_read sums the event intervals of the last sg_match by kernel
+ * class: 0 encoder, 1 q|k|v GEMM, 2 attention, 3 update-MLP layer 1 GEMM,
+ * 4 update-MLP layer 2 GEMM, 5 final projection GEMM, 6 score GEMM,
+ * 7 Sinkhorn + extraction.  ms_by_class and launches_by_class need n_classes
+ * >= 8 entries; returns the number of classes written, or -1.
+ */
+sg_status_t sg_profile(sg_handle* h, int enable);
+int sg_profile_read(sg_handle* h, float* ms_by_class, int* launches_by_class, int n_classes);
+
 /* Static description of a status code. */
 const char* sg_strerror(sg_status_t s);
 

@@ -25,7 +25,10 @@ STATUS = {0: "SG_OK", 1: "SG_ERR_INVALID_ARG", 2: "SG_ERR_SHAPE", 3: "SG_ERR_OOM
 
 EXPORTED = ["sg_create", "sg_destroy", "sg_match", "sg_match_host", "sg_scores",
             "sg_optimal_transport", "sg_status", "sg_strerror", "sg_launches_per_match",
-            "sg_selftest_barrier_timeout"]
+            "sg_selftest_barrier_timeout", "sg_profile", "sg_profile_read"]
+
+KERNEL_CLASSES = ["encoder", "qkv_gemm", "attention", "mlp1_gemm", "mlp2_gemm", "proj_gemm",
+                  "score_gemm", "sinkhorn"]
 
 _FP = C.POINTER(C.c_float)
 
@@ -95,6 +98,10 @@ def load():
     lib.sg_launches_per_match.restype = i32
     lib.sg_selftest_barrier_timeout.argtypes = [vp, C.c_uint, vp]
     lib.sg_selftest_barrier_timeout.restype = i32
+    lib.sg_profile.argtypes = [vp, i32]
+    lib.sg_profile.restype = i32
+    lib.sg_profile_read.argtypes = [vp, C.POINTER(C.c_float), C.POINTER(C.c_int), i32]
+    lib.sg_profile_read.restype = i32
     _lib = lib
     return lib
 
@@ -207,6 +214,18 @@ class Matcher:
 
     def selftest_barrier_timeout(self, timeout_us=20000, stream=None):
         return self.lib.sg_selftest_barrier_timeout(self.h, timeout_us, _stream_ptr(stream))
+
+    def profile(self, enable: bool):
+        _check(self.lib.sg_profile(self.h, 1 if enable else 0), "sg_profile")
+
+    def profile_read(self):
+        """{class: (ms, launches)} of the last sg_match (stream must be synchronised)."""
+        n = len(KERNEL_CLASSES)
+        ms = (C.c_float * n)()
+        cnt = (C.c_int * n)()
+        if self.lib.sg_profile_read(self.h, ms, cnt, n) < 0:
+            raise SgError(4, "sg_profile_read")
+        return {KERNEL_CLASSES[i]: (float(ms[i]), int(cnt[i])) for i in range(n)}
 
     def launches_per_match(self, B, M, N):
         return self.lib.sg_launches_per_match(self.h, B, M, N)

@@ -81,6 +81,11 @@ struct sg_handle {
   cudaGraphExec_t gexec;
   std::vector<void*> allocs;
   sg_status_t sticky;
+  // per-kernel timing (events between launches, also captured into graphs)
+  bool profiling;
+  std::vector<cudaEvent_t> prof_ev;
+  std::vector<int> prof_cls;
+  int prof_n;
 };
 
 namespace {
@@ -89,6 +94,17 @@ sg_status_t cuda_err(sg_handle* h, cudaError_t e) {
   if (e == cudaSuccess) return SG_OK;
   if (h) h->sticky = SG_ERR_CUDA;
   return SG_ERR_CUDA;
+}
+
+// Kernel classes of the per-kernel timing (sg_profile_read).
+enum KClass { K_ENCODER = 0, K_QKV, K_ATTN, K_MLP1, K_MLP2, K_PROJ, K_SCORE, K_SINKHORN, K_END };
+
+void mark(sg_handle* h, cudaStream_t s, int cls) {
+  if (!h->profiling) return;
+  if (h->prof_n >= (int)h->prof_ev.size()) return;
+  cudaEventRecordWithFlags(h->prof_ev[h->prof_n], s, cudaEventRecordExternal);
+  h->prof_cls[h->prof_n] = cls;
+  ++h->prof_n;
 }
 
 // ---------------------------------------------------------------- weight folding
@@ -220,7 +236,8 @@ struct Inputs {
 };
 
 cudaError_t gemm(sg_handle* h, const GemmArgs& g, int epi, bool out_bf16, int batch, cudaStream_t s,
-                 int* launches) {
+                 int* launches, int cls) {
+  mark(h, s, cls);
   ++*launches;
   if (h->use_tc) return launch_gemm_tc(g, epi, batch, s);
   return launch_gemm_simt(g, epi, h->bf16, out_bf16, batch, s);
@@ -245,6 +262,7 @@ cudaError_t run_network(sg_handle* h, int B, int M, int N, const Inputs& in, flo
   ea.cy = c.img_h * 0.5f;
   const float mx = c.img_w > c.img_h ? c.img_w : c.img_h;
   ea.inv_scale = (float)(1.0 / (c.norm_mode == 0 ? 0.7 * (double)mx : 0.5 * (double)mx));
+  mark(h, s, K_ENCODER);
   cudaError_t e = launch_encoder(ea, h->bf16, s);
   ++*launches;
   if (e != cudaSuccess) return e;
@@ -256,11 +274,12 @@ cudaError_t run_network(sg_handle* h, int B, int M, int N, const Inputs& in, flo
     g.A0 = xin; g.A1 = nullptr; g.lda = kD; g.k_split = kD;
     g.W = w.Wqkv; g.bias = w.bqkv; g.out = h->qkv; g.ldo = kQKV;
     g.rows = R; g.cols = kQKV; g.K = kD; g.scale = 1.f;
-    if ((e = gemm(h, g, EPI_BIAS, h->bf16, 1, s, launches)) != cudaSuccess) return e;
+    if ((e = gemm(h, g, EPI_BIAS, h->bf16, 1, s, launches, K_QKV)) != cudaSuccess) return e;
     AttnArgs aa{};
     aa.qkv = h->qkv; aa.msg = h->msg; aa.B = B; aa.M = M; aa.N = N;
     aa.cross = (st % 2 == 1);
     aa.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)kDh));
+    mark(h, s, K_ATTN);
     ++*launches;
     e = h->use_tc ? launch_attention_tc(aa, s) : launch_attention_simt(aa, h->bf16, s);
     if (e != cudaSuccess) return e;
@@ -269,20 +288,20 @@ cudaError_t run_network(sg_handle* h, int B, int M, int N, const Inputs& in, flo
     g.A0 = xin; g.A1 = h->msg; g.lda = kD; g.k_split = kD;
     g.W = w.W1; g.bias = w.b1; g.out = h->hid; g.ldo = 2 * kD;
     g.rows = R; g.cols = 2 * kD; g.K = 2 * kD; g.scale = 1.f;
-    if ((e = gemm(h, g, EPI_BIAS_RELU, h->bf16, 1, s, launches)) != cudaSuccess) return e;
+    if ((e = gemm(h, g, EPI_BIAS_RELU, h->bf16, 1, s, launches, K_MLP1)) != cudaSuccess) return e;
     // x += W2 h   (bias 0), refresh the bf16 shadow
     g = GemmArgs{};
     g.A0 = h->hid; g.A1 = nullptr; g.lda = 2 * kD; g.k_split = 2 * kD;
     g.W = w.W2; g.bias = nullptr; g.out = h->x32; g.out2 = h->x16; g.ldo = kD;
     g.rows = R; g.cols = kD; g.K = 2 * kD; g.scale = 1.f;
-    if ((e = gemm(h, g, EPI_RESIDUAL, h->bf16, 1, s, launches)) != cudaSuccess) return e;
+    if ((e = gemm(h, g, EPI_RESIDUAL, h->bf16, 1, s, launches, K_MLP2)) != cudaSuccess) return e;
   }
   // f = Wf x + bf
   GemmArgs g{};
   g.A0 = xin; g.A1 = nullptr; g.lda = kD; g.k_split = kD;
   g.W = h->Wf; g.bias = h->bf; g.out = h->f; g.ldo = kD;
   g.rows = R; g.cols = kD; g.K = kD; g.scale = 1.f;
-  if ((e = gemm(h, g, EPI_BIAS, h->bf16, 1, s, launches)) != cudaSuccess) return e;
+  if ((e = gemm(h, g, EPI_BIAS, h->bf16, 1, s, launches, K_PROJ)) != cudaSuccess) return e;
   // S_b = f_A f_B^T / sqrt(D), batched over pairs
   g = GemmArgs{};
   g.A0 = h->f; g.A1 = nullptr; g.lda = kD; g.k_split = kD;
@@ -291,7 +310,7 @@ cudaError_t run_network(sg_handle* h, int B, int M, int N, const Inputs& in, flo
   g.rows = M; g.cols = N; g.K = kD;
   g.strideA = (long long)P * kD; g.strideW = (long long)P * kD; g.strideO = strideS;
   g.scale = (float)(1.0 / std::sqrt((double)kD));
-  return gemm(h, g, EPI_SCALE, false, B, s, launches);
+  return gemm(h, g, EPI_SCALE, false, B, s, launches, K_SCORE);
 }
 
 // Steps 4-5 from S.
@@ -319,6 +338,7 @@ cudaError_t run_transport(sg_handle* h, int B, int M, int N, const float* S, lon
   off += (size_t)B * M * 4;
   off = (off + 255) & ~(size_t)255;
   a.max0 = reinterpret_cast<float*>(p + off);
+  mark(h, st, K_SINKHORN);
   cudaError_t e = cudaMemsetAsync(p, 0, zero_bytes, st);
   if (e != cudaSuccess) return e;
   a.S = S; a.lds = lds; a.strideS = strideS; a.alpha = h->alpha;
@@ -327,7 +347,9 @@ cudaError_t run_transport(sg_handle* h, int B, int M, int N, const float* S, lon
   a.logP = logP; a.matches0 = m0; a.matches1 = m1; a.mscores0 = s0; a.mscores1 = s1;
   a.status = h->status;
   a.timeout_ns = 1000000000ull;   // 1 s per barrier wait
-  return launch_sinkhorn(a, h->num_sms, st, launches);
+  e = launch_sinkhorn(a, h->num_sms, st, launches);
+  mark(h, st, K_END);
+  return e;
 }
 
 sg_status_t check_shape(sg_handle* h, int B, int M, int N) {
@@ -489,6 +511,7 @@ void sg_destroy(sg_handle* h) {
   cudaDeviceSynchronize();
   if (h->graph_valid) cudaGraphExecDestroy(h->gexec);
   if (h->cap_stream) cudaStreamDestroy(h->cap_stream);
+  for (cudaEvent_t ev : h->prof_ev) cudaEventDestroy(ev);
   for (void* p : h->allocs) cudaFree(p);
   delete h;
 }
@@ -537,11 +560,12 @@ sg_status_t sg_match(sg_handle* h, int B, int M, int N, const float* kpts0, cons
   const long long strideS = (long long)M * lds;
   Inputs in{kpts0, conf0, desc0, kpts1, conf1, desc1};
   GraphKey key{};
-  key.B = B; key.M = M; key.N = N; key.kind = 1;
+  key.B = B; key.M = M; key.N = N; key.kind = h->profiling ? 2 : 1;
   const void* ps[12] = {kpts0, conf0, desc0, kpts1, conf1, desc1, out_logP, matches0, matches1,
                         mscores0, mscores1, nullptr};
   std::memcpy(key.p, ps, sizeof(ps));
   return run_maybe_graph(h, key, s, [&](cudaStream_t cs, int* launches) -> cudaError_t {
+    h->prof_n = 0;
     cudaError_t e = run_network(h, B, M, N, in, h->Z, lds, strideS, cs, launches);
     if (e != cudaSuccess) return e;
     return run_transport(h, B, M, N, h->Z, lds, strideS, out_logP, matches0, matches1, mscores0,
@@ -604,6 +628,35 @@ sg_status_t sg_selftest_barrier_timeout(sg_handle* h, unsigned timeout_us, void*
   if (e != cudaSuccess) return cuda_err(h, e);
   if (ret != 1) return SG_ERR_INVALID_ARG;   // the wait did not report its expiry
   return sg_status(h, stream);
+}
+
+sg_status_t sg_profile(sg_handle* h, int enable) {
+  if (!h) return SG_ERR_INVALID_ARG;
+  if (enable && h->prof_ev.empty()) {
+    const int n = 8 + 4 * h->cfg.n_stages + 4;
+    h->prof_ev.resize(n);
+    h->prof_cls.assign(n, -1);
+    for (int i = 0; i < n; ++i)
+      if (cudaEventCreate(&h->prof_ev[i]) != cudaSuccess) return cuda_err(h, cudaGetLastError());
+  }
+  h->profiling = enable != 0;
+  h->prof_n = 0;
+  return SG_OK;
+}
+
+int sg_profile_read(sg_handle* h, float* ms_by_class, int* launches_by_class, int n_classes) {
+  if (!h || !ms_by_class || !launches_by_class || n_classes < K_END) return -1;
+  for (int c = 0; c < n_classes; ++c) { ms_by_class[c] = 0.f; launches_by_class[c] = 0; }
+  for (int i = 0; i + 1 < h->prof_n; ++i) {
+    float ms = 0.f;
+    if (cudaEventElapsedTime(&ms, h->prof_ev[i], h->prof_ev[i + 1]) != cudaSuccess) {
+      cudaGetLastError();
+      return -1;
+    }
+    const int c = h->prof_cls[i];
+    if (c >= 0 && c < K_END) { ms_by_class[c] += ms; launches_by_class[c] += 1; }
+  }
+  return K_END;
 }
 
 sg_status_t sg_status(sg_handle* h, void* stream) {
