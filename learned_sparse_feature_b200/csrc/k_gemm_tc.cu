@@ -1,9 +1,327 @@
-// tcgen05 (5th-generation tensor core) kernels: placeholder until the sm_100a
-// GEMM and attention kernels land.
+// tcgen05 GEMM with fused epilogues: every linear layer of the bf16 path (q|k|v
+// projection, the two update-MLP layers with folded BatchNorm + ReLU and the
+// residual add, the final projection) and the batched score matrix
+// S = <f_A, f_B> / sqrt(D) ("笔记：SuperGlue:Learning Feature Matching with Graph
+// Neural Networks论文阅读", sections 多层GNN and 匹配得分预测).
+//
+// C[128 x BN tile] = A[rows x K] * W[cols x K]^T, both operands K-major bf16.
+// One CTA of 4 warps per output tile:
+//   warp 0 (one lane)  TMA producer: 128x64 A and BNx64 W tiles per K-block,
+//                      128-byte swizzle, STAGES-deep ring of shared buffers;
+//   warp 1 (one lane)  MMA issuer: 4 x tcgen05.mma (K = 16 each) per K-block into
+//                      a 128 x BN fp32 accumulator in TMEM, tcgen05.commit frees
+//                      the stage;
+//   warps 0-3          epilogue: tcgen05.ld of the thread's accumulator row (TMEM
+//                      lane = tile row), bias / ReLU / residual / scale, store.
+// The A operand may come from two tensors split along K (the update MLP reads
+// [x || message] without materialising the concatenation).
 #include "sg_internal.cuh"
+#include "tc_common.cuh"
+
+#include <cudaTypedefs.h>
+
+#include <mutex>
 
 namespace sg {
-bool tc_available() { return false; }
-cudaError_t launch_gemm_tc(const GemmArgs&, int, int, cudaStream_t) { return cudaErrorNotSupported; }
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;                   // one 128-byte swizzle atom of bf16
+constexpr int kThreads = 128;
+constexpr unsigned kErrGemmWait = 4u;    // status bit: a GEMM pipeline wait ran out
+
+struct TcArgs {
+  int rows, cols, K, k_split;
+  int a_batch_rows;      // row offset between batches in the A tensor
+  int b_batch_rows;      // row offset between batches in the W tensor
+  int b_row0;            // first W row of batch 0
+  const float* bias;
+  void* out;
+  void* out2;
+  long long ldo;
+  long long strideO;
+  float scale;
+  unsigned* status;
+};
+
+template <int BN, int STAGES>
+struct Smem {
+  static constexpr int A_BYTES = BM * BK * 2;
+  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int BYTES = STAGES * STAGE_BYTES + 1024;   // + alignment slack
+};
+
+template <int BN> __host__ __device__ constexpr uint32_t tmem_cols() {
+  return BN <= 32 ? 32 : BN <= 64 ? 64 : BN <= 128 ? 128 : 256;
+}
+
+template <int BN, int STAGES, int EPI>
+__global__ void __launch_bounds__(kThreads, 1)
+gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
+               const __grid_constant__ CUtensorMap tmB, TcArgs g) {
+  using SM = Smem<BN, STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t full_bar[STAGES];
+  __shared__ __align__(8) uint64_t empty_bar[STAGES];
+  __shared__ __align__(8) uint64_t accum_bar;
+  __shared__ uint32_t tmem_slot;
+  __shared__ int s_abort;
+
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  const uint32_t base = (tc::smem_u32(smem_raw) + 1023u) & ~1023u;
+  uint8_t* sbase = smem_raw + (base - tc::smem_u32(smem_raw));
+
+  const int bz = blockIdx.z;
+  const int m0 = blockIdx.y * BM;
+  const int n0 = blockIdx.x * BN;
+  const int a_row = bz * g.a_batch_rows + m0;
+  const int b_row = g.b_row0 + bz * g.b_batch_rows + n0;
+  const int nkb = g.K / BK;
+  const int nkb0 = g.k_split / BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      tc::mbar_init(&full_bar[s], 1);
+      tc::mbar_init(&empty_bar[s], 1);
+    }
+    tc::mbar_init(&accum_bar, 1);
+    tc::fence_barrier_init();
+    s_abort = 0;
+  }
+  if (warp == 0) {
+    tc::tmem_alloc(&tmem_slot, tmem_cols<BN>());
+  }
+  if (threadIdx.x == 32) {
+    tc::prefetch_tmap(&tmA0);
+    tc::prefetch_tmap(&tmA1);
+    tc::prefetch_tmap(&tmB);
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    // ---------------- TMA producer
+    int issued = 0;
+    for (int kb = 0; kb < nkb; ++kb) {
+      const int s = kb % STAGES;
+      const int round = kb / STAGES;
+      if (round > 0 && !tc::mbar_wait(&empty_bar[s], (round - 1) & 1, g.status, kErrGemmWait)) {
+        s_abort = 1;
+        break;
+      }
+      uint8_t* sa = sbase + s * SM::STAGE_BYTES;
+      uint8_t* sb = sa + SM::A_BYTES;
+      tc::mbar_arrive_expect_tx(&full_bar[s], SM::STAGE_BYTES);
+      if (kb < nkb0) tc::tma_load_2d(&tmA0, &full_bar[s], sa, kb * BK, a_row);
+      else tc::tma_load_2d(&tmA1, &full_bar[s], sa, (kb - nkb0) * BK, a_row);
+      tc::tma_load_2d(&tmB, &full_bar[s], sb, kb * BK, b_row);
+      ++issued;
+    }
+    // drain: the copies in flight must land before the CTA may exit
+    for (int kb = (issued > STAGES ? issued - STAGES : 0); kb < issued; ++kb)
+      tc::mbar_wait(&full_bar[kb % STAGES], (kb / STAGES) & 1, g.status, kErrGemmWait);
+  } else if (warp == 1 && lane == 0) {
+    // ---------------- MMA issuer
+    constexpr uint32_t idesc = tc::idesc_bf16_f32(BM, BN);
+    bool ok = true;
+    for (int kb = 0; kb < nkb; ++kb) {
+      const int s = kb % STAGES;
+      if (!tc::mbar_wait(&full_bar[s], (kb / STAGES) & 1, g.status, kErrGemmWait)) {
+        ok = false;
+        break;
+      }
+      tc::tc_fence_after();
+      const uint32_t sa = base + s * SM::STAGE_BYTES;
+      const uint32_t sb = sa + SM::A_BYTES;
+      const uint64_t da = tc::sdesc_k_sw128(sa);
+      const uint64_t db = tc::sdesc_k_sw128(sb);
+#pragma unroll
+      for (int kk = 0; kk < BK / 16; ++kk)   // +32 B along K inside the swizzle atom
+        tc::umma_bf16(tmem, da + 2 * kk, db + 2 * kk, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+      tc::umma_commit(&empty_bar[s]);
+    }
+    if (ok) tc::umma_commit(&accum_bar);
+    else { s_abort = 1; tc::mbar_arrive(&accum_bar); }
+  }
+  __syncwarp();
+
+  // ---------------- epilogue: thread t owns tile row t (TMEM lane t)
+  const bool have = tc::mbar_wait(&accum_bar, 0, g.status, kErrGemmWait);
+  tc::tc_fence_after();
+  const int row = m0 + threadIdx.x;
+  const bool row_ok = have && row < g.rows && !s_abort;
+  const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+#pragma unroll 1
+  for (int c0 = 0; c0 < BN; c0 += 32) {
+    float v[32];
+    tc::tmem_ld32(trow + c0, v);        // warp-collective: every lane takes part
+    if (!row_ok || n0 + c0 >= g.cols) continue;
+    const long long obase = (long long)bz * g.strideO + (long long)row * g.ldo + n0 + c0;
+    const int ncol = min(32, g.cols - (n0 + c0));
+    if (EPI == EPI_BIAS || EPI == EPI_BIAS_RELU) {
+      __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(g.out) + obase;
+      if (ncol == 32) {
+        uint4 pk[4];
+        uint32_t* p = reinterpret_cast<uint32_t*>(pk);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          float a = v[2 * i] + __ldg(g.bias + n0 + c0 + 2 * i);
+          float b = v[2 * i + 1] + __ldg(g.bias + n0 + c0 + 2 * i + 1);
+          if (EPI == EPI_BIAS_RELU) { a = fmaxf(a, 0.f); b = fmaxf(b, 0.f); }
+          p[i] = tc::pack_bf16x2(a, b);
+        }
+        uint4* o4 = reinterpret_cast<uint4*>(o);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) o4[i] = pk[i];
+      } else {
+        for (int i = 0; i < ncol; ++i) {
+          float a = v[i] + g.bias[n0 + c0 + i];
+          if (EPI == EPI_BIAS_RELU) a = fmaxf(a, 0.f);
+          o[i] = __float2bfloat16_rn(a);
+        }
+      }
+    } else if (EPI == EPI_RESIDUAL) {
+      float* x = reinterpret_cast<float*>(g.out) + obase;
+      __nv_bfloat16* xb = reinterpret_cast<__nv_bfloat16*>(g.out2) + obase;
+      if (ncol == 32) {
+        float4* x4 = reinterpret_cast<float4*>(x);
+        uint4 pk[4];
+        uint32_t* p = reinterpret_cast<uint32_t*>(pk);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          float4 r = x4[i];
+          r.x += v[4 * i]; r.y += v[4 * i + 1]; r.z += v[4 * i + 2]; r.w += v[4 * i + 3];
+          x4[i] = r;
+          p[2 * i] = tc::pack_bf16x2(r.x, r.y);
+          p[2 * i + 1] = tc::pack_bf16x2(r.z, r.w);
+        }
+        uint4* o4 = reinterpret_cast<uint4*>(xb);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) o4[i] = pk[i];
+      } else {
+        for (int i = 0; i < ncol; ++i) {
+          const float r = x[i] + v[i];
+          x[i] = r;
+          xb[i] = __float2bfloat16_rn(r);
+        }
+      }
+    } else {
+      float* o = reinterpret_cast<float*>(g.out) + obase;
+      for (int i = 0; i < ncol; ++i) o[i] = v[i] * g.scale;
+    }
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tc::tmem_dealloc(tmem, tmem_cols<BN>());
+}
+
+// ------------------------------------------------------------------ host side
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// Row-major bf16 matrix [rows x cols] (row stride ld elements), boxes of
+// box_rows x 64 with the 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* ptr, long long rows, long long cols, long long ld, int box_rows) {
+  auto enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)(ld * 2)};
+  cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int BN, int STAGES, int EPI>
+cudaError_t launch_t(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b, const TcArgs& t,
+                     dim3 grid, cudaStream_t s) {
+  auto kern = gemm_tc_kernel<BN, STAGES, EPI>;
+  constexpr int smem = Smem<BN, STAGES>::BYTES;
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  kern<<<grid, kThreads, smem, s>>>(a0, a1, b, t);
+  return cudaGetLastError();
+}
+
+template <int BN, int STAGES>
+cudaError_t launch_epi(int epi, const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b,
+                       const TcArgs& t, dim3 grid, cudaStream_t s) {
+  switch (epi) {
+    case EPI_BIAS: return launch_t<BN, STAGES, EPI_BIAS>(a0, a1, b, t, grid, s);
+    case EPI_BIAS_RELU: return launch_t<BN, STAGES, EPI_BIAS_RELU>(a0, a1, b, t, grid, s);
+    case EPI_RESIDUAL: return launch_t<BN, STAGES, EPI_RESIDUAL>(a0, a1, b, t, grid, s);
+    default: return launch_t<BN, STAGES, EPI_SCALE>(a0, a1, b, t, grid, s);
+  }
+}
+
+}  // namespace
+
+bool tc_available() { return get_encode() != nullptr; }
+
+// GemmArgs (shared with the CUDA-core path) -> tensor maps + tcgen05 launch.
+// Requirements: K and k_split multiples of 64, lda/ldo multiples of 8 elements.
+cudaError_t launch_gemm_tc(const GemmArgs& g, int epi, int batch, cudaStream_t s, unsigned* status) {
+  if (g.rows <= 0 || g.cols <= 0 || batch <= 0) return cudaSuccess;
+  if (g.K % BK || g.k_split % BK || g.lda % 8) return cudaErrorInvalidValue;
+  // Column tile: wide enough to amortise the A tile, narrow enough to fill the SMs.
+  int BN;
+  const long long row_tiles = (long long)((g.rows + BM - 1) / BM) * batch;
+  if (epi == EPI_SCALE) BN = 128;
+  else if (g.cols % 256 == 0 && row_tiles * (g.cols / 256) >= 148) BN = 256;
+  else if (g.cols % 128 == 0 && row_tiles * (g.cols / 128) >= 120) BN = 128;
+  else if (g.cols % 64 == 0) BN = 64;
+  else BN = 128;
+  // A rows: rows of one batch item live at strideA / lda rows apart
+  const long long a_batch_rows = batch > 1 ? g.strideA / g.lda : 0;
+  const long long b_batch_rows = batch > 1 ? g.strideW / g.K : 0;
+  const long long a_total_rows = batch > 1 ? a_batch_rows * (batch - 1) + g.rows : g.rows;
+  CUtensorMap a0, a1, b;
+  if (!make_map(&a0, g.A0, a_total_rows, g.k_split, g.lda, BM)) return cudaErrorInvalidValue;
+  if (g.A1) {
+    if (!make_map(&a1, g.A1, a_total_rows, g.K - g.k_split, g.lda, BM)) return cudaErrorInvalidValue;
+  } else {
+    a1 = a0;
+  }
+  // For the batched score GEMM W is a row window of a taller matrix (f_B rows);
+  // map the whole window of all batches.
+  const long long b_total_rows = batch > 1 ? b_batch_rows * (batch - 1) + g.cols : g.cols;
+  if (!make_map(&b, g.W, b_total_rows, g.K, g.K, BN)) return cudaErrorInvalidValue;
+  TcArgs t{};
+  t.rows = g.rows; t.cols = g.cols; t.K = g.K; t.k_split = g.k_split;
+  t.a_batch_rows = (int)a_batch_rows;
+  t.b_batch_rows = (int)b_batch_rows;
+  t.b_row0 = 0;
+  t.bias = g.bias; t.out = g.out; t.out2 = g.out2; t.ldo = g.ldo; t.strideO = g.strideO;
+  t.scale = g.scale; t.status = status;
+  dim3 grid((g.cols + BN - 1) / BN, (g.rows + BM - 1) / BM, batch);
+  switch (BN) {
+    case 256: return launch_epi<256, 3>(epi, a0, a1, b, t, grid, s);
+    case 128: return launch_epi<128, 4>(epi, a0, a1, b, t, grid, s);
+    default: return launch_epi<64, 6>(epi, a0, a1, b, t, grid, s);
+  }
+}
+
 cudaError_t launch_attention_tc(const AttnArgs&, cudaStream_t) { return cudaErrorNotSupported; }
+
 }  // namespace sg

@@ -51,7 +51,8 @@ struct sg_handle {
   int device;
   int num_sms;
   bool bf16;
-  bool use_tc;
+  bool use_tc;        // tcgen05 GEMMs
+  bool use_tc_attn;   // tcgen05 attention
   // weights
   float* encW[SG_ENC_LAYERS];
   float* encb[SG_ENC_LAYERS];
@@ -239,7 +240,7 @@ cudaError_t gemm(sg_handle* h, const GemmArgs& g, int epi, bool out_bf16, int ba
                  int* launches, int cls) {
   mark(h, s, cls);
   ++*launches;
-  if (h->use_tc) return launch_gemm_tc(g, epi, batch, s);
+  if (h->use_tc) return launch_gemm_tc(g, epi, batch, s, h->status);
   return launch_gemm_simt(g, epi, h->bf16, out_bf16, batch, s);
 }
 
@@ -281,7 +282,7 @@ cudaError_t run_network(sg_handle* h, int B, int M, int N, const Inputs& in, flo
     aa.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)kDh));
     mark(h, s, K_ATTN);
     ++*launches;
-    e = h->use_tc ? launch_attention_tc(aa, s) : launch_attention_simt(aa, h->bf16, s);
+    e = h->use_tc_attn ? launch_attention_tc(aa, s) : launch_attention_simt(aa, h->bf16, s);
     if (e != cudaSuccess) return e;
     // h = relu(W1' [x || m] + b1')
     g = GemmArgs{};
@@ -462,6 +463,7 @@ sg_status_t sg_create(const sg_weights* w, const sg_config* cfg, sg_handle** out
   h->num_sms = prop.multiProcessorCount;
   h->bf16 = cfg->precision == SG_PRECISION_BF16;
   h->use_tc = h->bf16 && tc_available() && std::getenv("SG_FORCE_SIMT") == nullptr;
+  h->use_tc_attn = false;
   h->use_graph = std::getenv("SG_NO_GRAPH") == nullptr;
   h->sticky = SG_OK;
   sg_status_t st = pack_weights(h, w);
@@ -670,7 +672,7 @@ sg_status_t sg_status(sg_handle* h, void* stream) {
   sg_status_t sticky = h->sticky;
   h->sticky = SG_OK;
   if (sticky != SG_OK) return sticky;
-  if (word & kStatusTimeout) return SG_ERR_TIMEOUT;
+  if (word & (kStatusTimeout | kStatusPipeline)) return SG_ERR_TIMEOUT;
   if (word & kStatusNumeric) return SG_ERR_NUMERIC;
   return SG_OK;
 }

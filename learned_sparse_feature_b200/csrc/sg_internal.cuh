@@ -17,6 +17,7 @@ constexpr int kQKV = 3 * kD;   // fused q|k|v row width
 // Device status word bits (latched by kernels, read by sg_status).
 constexpr unsigned kStatusTimeout = 1u;
 constexpr unsigned kStatusNumeric = 2u;
+constexpr unsigned kStatusPipeline = 4u;   // a tcgen05 pipeline wait ran out
 
 // ------------------------------------------------------------------ GEMM epilogues
 enum Epilogue : int {
@@ -107,8 +108,8 @@ cudaError_t launch_barrier_selftest(unsigned* scratch, unsigned* status, unsigne
                                     int* returned, cudaStream_t s);
 
 // tcgen05 paths (sm_100a)
-struct TcGemm;   // opaque plan (tensor maps) built on the host
-cudaError_t launch_gemm_tc(const GemmArgs& g, int epi, int batch, cudaStream_t s);
+// status: device status word; a pipeline wait that runs out sets a bit in it.
+cudaError_t launch_gemm_tc(const GemmArgs& g, int epi, int batch, cudaStream_t s, unsigned* status);
 cudaError_t launch_attention_tc(const AttnArgs& a, cudaStream_t s);
 bool tc_available();
 

@@ -235,3 +235,24 @@ def test_non_finite_input_is_reported(dev, weights):
     m.optimal_transport(torch.from_numpy(S).to(dev), lp, *outs)
     assert m.status() == 6                              # SG_ERR_NUMERIC
     m.close()
+
+
+@pytest.mark.parametrize("B,M,N", [(1, 300, 200), (2, 128, 256), (3, 65, 190)])
+def test_tensor_core_path_matches_cuda_core_path(dev, weights, B, M, N, monkeypatch):
+    # same bf16 operands, fp32 accumulation in both: only the summation order differs
+    batch = _random_batch(B, M, N, seed=B * 1000 + M)
+    t = {k: torch.from_numpy(v).to(dev) for k, v in batch.items()}
+    out = []
+    for force_simt in (False, True):
+        if force_simt:
+            monkeypatch.setenv("SG_FORCE_SIMT", "1")
+        m = _matcher(weights, B, M, N, "bf16", n_stages=2)
+        S = torch.empty((B, M, N), device=dev)
+        m.scores(t["kpts0"], t["conf0"], t["desc0"], t["kpts1"], t["conf1"], t["desc1"], S)
+        assert m.status() == 0
+        out.append(S.double().cpu().numpy())
+        m.close()
+    assert np.abs(out[0] - out[1]).max() < 2e-2 * max(1.0, np.abs(out[1]).max() / 10)
+    for b in range(B):
+        ref = _oracle(batch, weights, b, n_stages=2)["scores"]
+        assert np.abs(out[0][b] - ref).max() < 5e-2
