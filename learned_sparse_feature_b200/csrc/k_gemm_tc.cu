@@ -234,9 +234,11 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
   return fn;
 }
 
+}  // namespace
+
 // Row-major bf16 matrix [rows x cols] (row stride ld elements), boxes of
 // box_rows x 64 with the 128-byte swizzle.
-bool make_map(CUtensorMap* m, const void* ptr, long long rows, long long cols, long long ld, int box_rows) {
+bool make_bf16_map(CUtensorMap* m, const void* ptr, long long rows, long long cols, long long ld, int box_rows) {
   auto enc = get_encode();
   if (!enc) return false;
   cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
@@ -248,6 +250,8 @@ bool make_map(CUtensorMap* m, const void* ptr, long long rows, long long cols, l
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
+
+namespace {
 
 template <int BN, int STAGES, int EPI>
 cudaError_t launch_t(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b, const TcArgs& t,
@@ -297,16 +301,16 @@ cudaError_t launch_gemm_tc(const GemmArgs& g, int epi, int batch, cudaStream_t s
   const long long b_batch_rows = batch > 1 ? g.strideW / g.K : 0;
   const long long a_total_rows = batch > 1 ? a_batch_rows * (batch - 1) + g.rows : g.rows;
   CUtensorMap a0, a1, b;
-  if (!make_map(&a0, g.A0, a_total_rows, g.k_split, g.lda, BM)) return cudaErrorInvalidValue;
+  if (!make_bf16_map(&a0, g.A0, a_total_rows, g.k_split, g.lda, BM)) return cudaErrorInvalidValue;
   if (g.A1) {
-    if (!make_map(&a1, g.A1, a_total_rows, g.K - g.k_split, g.lda, BM)) return cudaErrorInvalidValue;
+    if (!make_bf16_map(&a1, g.A1, a_total_rows, g.K - g.k_split, g.lda, BM)) return cudaErrorInvalidValue;
   } else {
     a1 = a0;
   }
   // For the batched score GEMM W is a row window of a taller matrix (f_B rows);
   // map the whole window of all batches.
   const long long b_total_rows = batch > 1 ? b_batch_rows * (batch - 1) + g.cols : g.cols;
-  if (!make_map(&b, g.W, b_total_rows, g.K, g.K, BN)) return cudaErrorInvalidValue;
+  if (!make_bf16_map(&b, g.W, b_total_rows, g.K, g.K, BN)) return cudaErrorInvalidValue;
   TcArgs t{};
   t.rows = g.rows; t.cols = g.cols; t.K = g.K; t.k_split = g.k_split;
   t.a_batch_rows = (int)a_batch_rows;
@@ -322,6 +326,5 @@ cudaError_t launch_gemm_tc(const GemmArgs& g, int epi, int batch, cudaStream_t s
   }
 }
 
-cudaError_t launch_attention_tc(const AttnArgs&, cudaStream_t) { return cudaErrorNotSupported; }
 
 }  // namespace sg

@@ -282,7 +282,7 @@ cudaError_t run_network(sg_handle* h, int B, int M, int N, const Inputs& in, flo
     aa.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)kDh));
     mark(h, s, K_ATTN);
     ++*launches;
-    e = h->use_tc_attn ? launch_attention_tc(aa, s) : launch_attention_simt(aa, h->bf16, s);
+    e = h->use_tc_attn ? launch_attention_tc(aa, s, h->status) : launch_attention_simt(aa, h->bf16, s);
     if (e != cudaSuccess) return e;
     // h = relu(W1' [x || m] + b1')
     g = GemmArgs{};
@@ -463,7 +463,7 @@ sg_status_t sg_create(const sg_weights* w, const sg_config* cfg, sg_handle** out
   h->num_sms = prop.multiProcessorCount;
   h->bf16 = cfg->precision == SG_PRECISION_BF16;
   h->use_tc = h->bf16 && tc_available() && std::getenv("SG_FORCE_SIMT") == nullptr;
-  h->use_tc_attn = false;
+  h->use_tc_attn = h->use_tc && std::getenv("SG_SIMT_ATTENTION") == nullptr;
   h->use_graph = std::getenv("SG_NO_GRAPH") == nullptr;
   h->sticky = SG_OK;
   sg_status_t st = pack_weights(h, w);

@@ -110,7 +110,7 @@ cudaError_t launch_barrier_selftest(unsigned* scratch, unsigned* status, unsigne
 // tcgen05 paths (sm_100a)
 // status: device status word; a pipeline wait that runs out sets a bit in it.
 cudaError_t launch_gemm_tc(const GemmArgs& g, int epi, int batch, cudaStream_t s, unsigned* status);
-cudaError_t launch_attention_tc(const AttnArgs& a, cudaStream_t s);
+cudaError_t launch_attention_tc(const AttnArgs& a, cudaStream_t s, unsigned* status);
 bool tc_available();
 
 }  // namespace sg

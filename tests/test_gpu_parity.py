@@ -256,3 +256,20 @@ def test_tensor_core_path_matches_cuda_core_path(dev, weights, B, M, N, monkeypa
     for b in range(B):
         ref = _oracle(batch, weights, b, n_stages=2)["scores"]
         assert np.abs(out[0][b] - ref).max() < 5e-2
+
+
+@pytest.mark.parametrize("B,M,N,cross_only", [(1, 300, 200, False), (2, 129, 257, False), (1, 1, 700, False)])
+def test_tensor_core_attention_matches_cuda_core_attention(dev, weights, B, M, N, cross_only, monkeypatch):
+    batch = _random_batch(B, M, N, seed=B * 77 + N)
+    t = {k: torch.from_numpy(v).to(dev) for k, v in batch.items()}
+    out = []
+    for simt in (False, True):
+        if simt:
+            monkeypatch.setenv("SG_SIMT_ATTENTION", "1")
+        m = _matcher(weights, B, M, N, "bf16", n_stages=2)
+        S = torch.empty((B, M, N), device=dev)
+        m.scores(t["kpts0"], t["conf0"], t["desc0"], t["kpts1"], t["conf1"], t["desc1"], S)
+        assert m.status() == 0
+        out.append(S.double().cpu().numpy())
+        m.close()
+    assert np.abs(out[0] - out[1]).max() < 2e-2 * max(1.0, np.abs(out[1]).max() / 10)
