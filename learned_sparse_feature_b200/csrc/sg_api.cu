@@ -325,8 +325,8 @@ cudaError_t run_transport(sg_handle* h, int B, int M, int N, const float* S, lon
   a.abort_flag = a.barrier + B;
   size_t off = ((B + 1) * sizeof(unsigned) + 255) & ~(size_t)255;
   a.acc = reinterpret_cast<float*>(p + off);
-  a.fb = a.acc + (size_t)B * 3 * C;
-  off += (size_t)B * 5 * C * 4;
+  a.fb = a.acc + (size_t)B * 3 * sinkhorn_acc_floats_per_buffer(N);
+  off += (size_t)B * 5 * sinkhorn_acc_floats_per_buffer(N) * 4;
   off = (off + 255) & ~(size_t)255;
   a.colbest = reinterpret_cast<unsigned long long*>(p + off);
   off += (size_t)B * N * 8;
@@ -343,6 +343,7 @@ cudaError_t run_transport(sg_handle* h, int B, int M, int N, const float* S, lon
   cudaError_t e = cudaMemsetAsync(p, 0, zero_bytes, st);
   if (e != cudaSuccess) return e;
   a.S = S; a.lds = lds; a.strideS = strideS; a.alpha = h->alpha;
+  a.lds_vec = (lds % 4 == 0) && (strideS % 4 == 0) && ((reinterpret_cast<uintptr_t>(S) & 15) == 0);
   a.B = B; a.M = M; a.N = N; a.iters = h->cfg.sinkhorn_iters;
   a.threshold = h->cfg.match_threshold;
   a.logP = logP; a.matches0 = m0; a.matches1 = m1; a.mscores0 = s0; a.mscores1 = s1;
@@ -450,7 +451,7 @@ sg_status_t sg_create(const sg_weights* w, const sg_config* cfg, sg_handle** out
       !(cfg->img_w > 0.f) || !(cfg->img_h > 0.f) || (cfg->norm_mode != 0 && cfg->norm_mode != 1) ||
       (cfg->precision != SG_PRECISION_FP32 && cfg->precision != SG_PRECISION_BF16))
     return SG_ERR_INVALID_ARG;
-  if (cfg->max_N + 1 > 16384) return SG_ERR_UNSUPPORTED;
+  if (cfg->max_N > 8192) return SG_ERR_UNSUPPORTED;   // Sinkhorn column slots per thread
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return SG_ERR_UNSUPPORTED; }
   cudaDeviceProp prop;
@@ -499,6 +500,7 @@ sg_status_t sg_create(const sg_weights* w, const sg_config* cfg, sg_handle** out
   h->s_ms0 = (float*)al(Bm * Mm * 4);
   h->s_ms1 = (float*)al(Bm * Nm * 4);
   if (!ok) { cudaGetLastError(); sg_destroy(h); return SG_ERR_OOM; }
+  if (sinkhorn_prepare(h->num_sms) != cudaSuccess) { cudaGetLastError(); sg_destroy(h); return SG_ERR_CUDA; }
   if (cudaMemset(h->status, 0, sizeof(unsigned)) != cudaSuccess ||
       cudaStreamCreateWithFlags(&h->cap_stream, cudaStreamNonBlocking) != cudaSuccess) {
     sg_destroy(h);
