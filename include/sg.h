@@ -114,8 +114,8 @@ typedef struct {
 } sg_weights;
 
 /*
- * Configuration.  The library supports D = 256 and H = 4 (d_head = 64); other
- * values return SG_ERR_UNSUPPORTED.  max_B/max_M/max_N size the workspace that
+ * Configuration.  The library supports D = 256 and H = 4 (d_head = 64), and
+ * max_N <= 3072; other values return SG_ERR_UNSUPPORTED.  max_B/max_M/max_N size the workspace that
  * the handle owns.  norm_mode 0 = (p - (W/2, H/2)) / (0.7 max(W, H)) as in the
  * Jazihars notes' normalize_keypoints; 1 = divide by max(W, H)/2 instead.
  */

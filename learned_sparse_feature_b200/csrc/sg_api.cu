@@ -451,7 +451,7 @@ sg_status_t sg_create(const sg_weights* w, const sg_config* cfg, sg_handle** out
       !(cfg->img_w > 0.f) || !(cfg->img_h > 0.f) || (cfg->norm_mode != 0 && cfg->norm_mode != 1) ||
       (cfg->precision != SG_PRECISION_FP32 && cfg->precision != SG_PRECISION_BF16))
     return SG_ERR_INVALID_ARG;
-  if (cfg->max_N > 8192) return SG_ERR_UNSUPPORTED;   // Sinkhorn column slots per thread
+  if (cfg->max_N > sinkhorn_max_columns()) return SG_ERR_UNSUPPORTED;   // transport kernel columns
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return SG_ERR_UNSUPPORTED; }
   cudaDeviceProp prop;

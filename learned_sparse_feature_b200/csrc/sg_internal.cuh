@@ -92,7 +92,7 @@ struct SinkhornArgs {
   unsigned* barrier;    // one counter per group
   unsigned* abort_flag;
   unsigned* status;
-  int team_clusters;    // clusters per team (set by the launcher)
+  int cpp;              // CTAs per pair group (set by the launcher)
   int band_alloc;       // rows per CTA band (set by the launcher)
   int lds_vec;          // S rows are 16-byte aligned (vector loads allowed)
   int cached_rows;      // rows of the band kept in shared memory
@@ -105,7 +105,8 @@ cudaError_t launch_gemm_simt(const GemmArgs& g, int epi, bool in_bf16, bool out_
                              int batch, cudaStream_t s);
 cudaError_t launch_attention_simt(const AttnArgs& a, bool bf16, cudaStream_t s);
 cudaError_t launch_sinkhorn(SinkhornArgs a, int num_sms, cudaStream_t s, int* launches);
-cudaError_t sinkhorn_prepare(int num_sms);   // attributes and residency queries (not capturable)
+cudaError_t sinkhorn_prepare(int num_sms);   // kernel attributes (called once, outside capture)
+int sinkhorn_max_columns();                  // largest N the transport kernel supports
 size_t sinkhorn_scratch_bytes(int B, int M, int N);
 size_t sinkhorn_acc_floats_per_buffer(int N);   // column accumulator floats per (pair, rotation)
 cudaError_t launch_barrier_selftest(unsigned* scratch, unsigned* status, unsigned long long timeout_ns,
