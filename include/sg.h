@@ -220,6 +220,32 @@ sg_status_t sg_selftest_barrier_timeout(sg_handle* h, unsigned timeout_us, void*
 sg_status_t sg_profile(sg_handle* h, int enable);
 int sg_profile_read(sg_handle* h, float* ms_by_class, int* launches_by_class, int n_classes);
 
+/*
+ * Steps 4-5 (transport + extraction, as sg_optimal_transport) for callers that
+ * cannot allocate device memory: a runtime without a device allocator, a plugin
+ * whose host application owns every allocation, or code running after memory
+ * was reserved up front.  No handle is needed and nothing is allocated: the
+ * scratch is a 4 MiB static device array inside the library, which every GPU
+ * that loads the library holds until the process exits.  The paper has no
+ * counterpart of this entry point; it exists for those callers.
+ *   scores: device B x M x N float32; outputs as for sg_match (out_logP may be
+ *   NULL); status: device word the caller zeroes, where device-side errors are
+ *   OR-ed in (1 = a bounded wait ran out, 2 = non-finite value).
+ * Returns SG_ERR_SHAPE if N > 3072 or the call needs more scratch than the
+ * static array holds (about 40 bytes per score-matrix column and per row of
+ * every pair).  The first call on a device does a one-time set-up (kernel
+ * attributes and the array's device address); make it before any stream
+ * capture.  Every call shares the one array and leaves its contents behind
+ * (the parts that must start at zero are cleared on the stream by each call),
+ * so calls that overlap on the GPU race: serialise them, e.g. on one stream.
+ */
+sg_status_t sg_optimal_transport_static(int B, int M, int N, const float* scores,
+                                        float bin_score, int sinkhorn_iters,
+                                        float match_threshold, float* out_logP,
+                                        int32_t* matches0, int32_t* matches1,
+                                        float* mscores0, float* mscores1,
+                                        unsigned* status, void* stream);
+
 /* Static description of a status code. */
 const char* sg_strerror(sg_status_t s);
 

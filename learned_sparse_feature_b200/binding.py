@@ -25,7 +25,8 @@ STATUS = {0: "SG_OK", 1: "SG_ERR_INVALID_ARG", 2: "SG_ERR_SHAPE", 3: "SG_ERR_OOM
 
 EXPORTED = ["sg_create", "sg_destroy", "sg_match", "sg_match_host", "sg_scores",
             "sg_optimal_transport", "sg_status", "sg_strerror", "sg_launches_per_match",
-            "sg_selftest_barrier_timeout", "sg_profile", "sg_profile_read"]
+            "sg_selftest_barrier_timeout", "sg_profile", "sg_profile_read",
+            "sg_optimal_transport_static"]
 
 KERNEL_CLASSES = ["encoder", "qkv_gemm", "attention", "mlp1_gemm", "mlp2_gemm", "proj_gemm",
                   "score_gemm", "sinkhorn"]
@@ -102,6 +103,8 @@ def load():
     lib.sg_profile.restype = i32
     lib.sg_profile_read.argtypes = [vp, C.POINTER(C.c_float), C.POINTER(C.c_int), i32]
     lib.sg_profile_read.restype = i32
+    lib.sg_optimal_transport_static.argtypes = [i32, i32, i32, vp, f32, i32, f32, vp, vp, vp, vp, vp, vp, vp]
+    lib.sg_optimal_transport_static.restype = i32
     _lib = lib
     return lib
 
@@ -229,6 +232,19 @@ class Matcher:
 
     def launches_per_match(self, B, M, N):
         return self.lib.sg_launches_per_match(self.h, B, M, N)
+
+
+def optimal_transport_static(scores, out_logP, matches0, matches1, mscores0, mscores1, status,
+                             bin_score=1.0, sinkhorn_iters=100, match_threshold=0.2, stream=None):
+    """sg_optimal_transport_static: transport + extraction without any device
+    allocation (library-owned static scratch).  Device tensors; `status` is a
+    zeroed int32 device tensor of one element that receives device-side errors."""
+    lib = load()
+    B, M, N = scores.shape
+    _check(lib.sg_optimal_transport_static(B, M, N, _ptr(scores), float(bin_score), int(sinkhorn_iters),
+                                           float(match_threshold), _ptr(out_logP), _ptr(matches0),
+                                           _ptr(matches1), _ptr(mscores0), _ptr(mscores1), _ptr(status),
+                                           _stream_ptr(stream)), "sg_optimal_transport_static")
 
 
 def match_batch(matcher: Matcher, batch: dict, with_logP: bool = True, stream=None):
