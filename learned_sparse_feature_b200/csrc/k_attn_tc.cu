@@ -18,6 +18,8 @@
 //                      K-major layout the MMA reads, and folds O_j into a running
 //                      fp32 output kept in registers (rescaled when the max grows).
 // The S MMA of tile j+1 overlaps the softmax of tile j.  Every wait is bounded.
+// Launched with programmatic dependent launch (prologue overlaps the previous
+// kernel; griddepcontrol.wait gates the first read of q|k|v).
 #include "sg_internal.cuh"
 #include "tc_common.cuh"
 
@@ -59,6 +61,9 @@ __device__ __forceinline__ float fast_ex2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -110,6 +115,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm, AttnTcArgs a) {
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = tmem_slot;
+  pdl_wait();                                    // q|k|v of the previous kernel are complete
 
   if (warp == 4) {
     if (lane == 0) {
@@ -167,6 +173,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm, AttnTcArgs a) {
         if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
       }
       if (ok) ok = issue_pv(ntiles - 1);
+      pdl_trigger();                             // no more tensor work: the next kernel may start
       if (!ok) s_abort = 1;
     }
   } else {
@@ -282,9 +289,17 @@ cudaError_t launch_attention_tc(const AttnArgs& a, cudaStream_t s, unsigned* sta
     attr = true;
   }
   AttnTcArgs t{reinterpret_cast<__nv_bfloat16*>(a.msg), a.B, a.M, a.N, a.cross, a.scale_log2, status};
-  dim3 grid((nmax + QT - 1) / QT, kH, 2 * a.B);
-  attn_tc_kernel<<<grid, kThreads, SMEM_BYTES, s>>>(tm, t);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((nmax + QT - 1) / QT, kH, 2 * a.B);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = SMEM_BYTES;
+  cfg.stream = s;
+  cudaLaunchAttribute la[1];
+  la[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // overlap with the previous kernel
+  la[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = la;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, attn_tc_kernel, tm, t);
 }
 
 }  // namespace sg

@@ -5,14 +5,18 @@
 // Neural Networks论文阅读", sections 多层GNN and 匹配得分预测).
 //
 // C[128 x BN tile] = A[rows x K] * W[cols x K]^T, both operands K-major bf16.
-// One CTA of 4 warps per output tile:
+// A persistent CTA of 6 warps loops over output tiles:
 //   warp 0 (one lane)  TMA producer: 128x64 A and BNx64 W tiles per K-block,
 //                      128-byte swizzle, STAGES-deep ring of shared buffers;
 //   warp 1 (one lane)  MMA issuer: 4 x tcgen05.mma (K = 16 each) per K-block into
-//                      a 128 x BN fp32 accumulator in TMEM, tcgen05.commit frees
-//                      the stage;
-//   warps 0-3          epilogue: tcgen05.ld of the thread's accumulator row (TMEM
-//                      lane = tile row), bias / ReLU / residual / scale, store.
+//                      one of two 128 x BN fp32 accumulators in TMEM;
+//                      tcgen05.commit frees the stage / publishes the tile;
+//   warps 2-5          epilogue: tcgen05.ld of the thread's accumulator row (TMEM
+//                      lane = tile row), bias / ReLU / residual / scale, store,
+//                      while the MMA warp already fills the other accumulator.
+// Launched with programmatic dependent launch: the prologue (barriers, TMEM,
+// descriptor prefetch) overlaps the previous kernel; griddepcontrol.wait gates
+// the first read of its outputs.
 // The A operand may come from two tensors split along K (the update MLP reads
 // [x || message] without materialising the concatenation).
 #include "sg_internal.cuh"
@@ -20,6 +24,7 @@
 
 #include <cudaTypedefs.h>
 
+#include <cmath>
 #include <mutex>
 
 namespace sg {
@@ -27,11 +32,11 @@ namespace {
 
 constexpr int BM = 128;
 constexpr int BK = 64;                   // one 128-byte swizzle atom of bf16
-constexpr int kThreads = 128;
+constexpr int kThreads = 192;                // producer, MMA, 4 epilogue warps
 constexpr unsigned kErrGemmWait = 4u;    // status bit: a GEMM pipeline wait ran out
 
 struct TcArgs {
-  int rows, cols, K, k_split;
+  int rows, cols, K, k_split, batch;
   int a_batch_rows;      // row offset between batches in the A tensor
   int b_batch_rows;      // row offset between batches in the W tensor
   int b_row0;            // first W row of batch 0
@@ -56,15 +61,25 @@ template <int BN> __host__ __device__ constexpr uint32_t tmem_cols() {
   return BN <= 32 ? 32 : BN <= 64 ? 64 : BN <= 128 ? 128 : 256;
 }
 
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// Persistent: CTA c computes output tiles c, c + gridDim.x, ...; tiles are
+// ordered (batch, row tile, column tile) with the column tile fastest so
+// consecutive CTAs share the A tile in L2.  The accumulator is double-buffered
+// in TMEM: the epilogue warps drain tile i while the MMA warp accumulates tile
+// i + 1.
 template <int BN, int STAGES, int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
                const __grid_constant__ CUtensorMap tmB, TcArgs g) {
   using SM = Smem<BN, STAGES>;
+  constexpr uint32_t BNA = tmem_cols<BN>();      // TMEM columns of one accumulator buffer
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[STAGES];
   __shared__ __align__(8) uint64_t empty_bar[STAGES];
-  __shared__ __align__(8) uint64_t accum_bar;
+  __shared__ __align__(8) uint64_t tfull_bar[2];
+  __shared__ __align__(8) uint64_t tempty_bar[2];
   __shared__ uint32_t tmem_slot;
   __shared__ int s_abort;
 
@@ -73,11 +88,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
   const uint32_t base = (tc::smem_u32(smem_raw) + 1023u) & ~1023u;
   uint8_t* sbase = smem_raw + (base - tc::smem_u32(smem_raw));
 
-  const int bz = blockIdx.z;
-  const int m0 = blockIdx.y * BM;
-  const int n0 = blockIdx.x * BN;
-  const int a_row = bz * g.a_batch_rows + m0;
-  const int b_row = g.b_row0 + bz * g.b_batch_rows + n0;
+  const int ntn = (g.cols + BN - 1) / BN;
+  const int ntm = (g.rows + BM - 1) / BM;
+  const int ntiles = ntn * ntm * g.batch;
   const int nkb = g.K / BK;
   const int nkb0 = g.k_split / BK;
 
@@ -86,14 +99,15 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
       tc::mbar_init(&full_bar[s], 1);
       tc::mbar_init(&empty_bar[s], 1);
     }
-    tc::mbar_init(&accum_bar, 1);
+    for (int b = 0; b < 2; ++b) {
+      tc::mbar_init(&tfull_bar[b], 1);
+      tc::mbar_init(&tempty_bar[b], 4);          // one arrival per epilogue warp
+    }
     tc::fence_barrier_init();
     s_abort = 0;
   }
-  if (warp == 0) {
-    tc::tmem_alloc(&tmem_slot, tmem_cols<BN>());
-  }
-  if (threadIdx.x == 32) {
+  if (warp == 1) tc::tmem_alloc(&tmem_slot, 2 * BNA);
+  if (threadIdx.x == 64) {
     tc::prefetch_tmap(&tmA0);
     tc::prefetch_tmap(&tmA1);
     tc::prefetch_tmap(&tmB);
@@ -102,121 +116,166 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = tmem_slot;
+  pdl_wait();                                    // the previous kernel's outputs are complete
 
-  if (warp == 0 && lane == 0) {
-    // ---------------- TMA producer
-    int issued = 0;
-    for (int kb = 0; kb < nkb; ++kb) {
-      const int s = kb % STAGES;
-      const int round = kb / STAGES;
-      if (round > 0 && !tc::mbar_wait(&empty_bar[s], (round - 1) & 1, g.status, kErrGemmWait)) {
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer
+      int it = 0;
+      for (int t = blockIdx.x; t < ntiles && !s_abort; t += gridDim.x) {
+        const int tn = t % ntn, tm = (t / ntn) % ntm, bz = t / (ntn * ntm);
+        const int a_row = bz * g.a_batch_rows + tm * BM;
+        const int b_row = g.b_row0 + bz * g.b_batch_rows + tn * BN;
+        for (int kb = 0; kb < nkb; ++kb, ++it) {
+          const int s = it % STAGES;
+          const int round = it / STAGES;
+          if (round > 0 && !tc::mbar_wait(&empty_bar[s], (round - 1) & 1, g.status, kErrGemmWait)) {
+            s_abort = 1;
+            break;
+          }
+          uint8_t* sa = sbase + s * SM::STAGE_BYTES;
+          uint8_t* sb = sa + SM::A_BYTES;
+          tc::mbar_arrive_expect_tx(&full_bar[s], SM::STAGE_BYTES);
+          if (kb < nkb0) tc::tma_load_2d(&tmA0, &full_bar[s], sa, kb * BK, a_row);
+          else tc::tma_load_2d(&tmA1, &full_bar[s], sa, (kb - nkb0) * BK, a_row);
+          tc::tma_load_2d(&tmB, &full_bar[s], sb, kb * BK, b_row);
+        }
+      }
+      // drain: copies in flight must land before the CTA may exit
+      for (int k = (it > STAGES ? it - STAGES : 0); k < it; ++k)
+        tc::mbar_wait(&full_bar[k % STAGES], (k / STAGES) & 1, g.status, kErrGemmWait);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer
+      constexpr uint32_t idesc = tc::idesc_bf16_f32(BM, BN);
+      int it = 0, i = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++i) {
+        const int b = i & 1;
+        if (i >= 2 && !tc::mbar_wait(&tempty_bar[b], ((i >> 1) - 1) & 1, g.status, kErrGemmWait)) {
+          ok = false;
+          break;
+        }
+        tc::tc_fence_after();
+        const uint32_t acc = tmem + b * BNA;
+        for (int kb = 0; kb < nkb; ++kb, ++it) {
+          const int s = it % STAGES;
+          if (!tc::mbar_wait(&full_bar[s], (it / STAGES) & 1, g.status, kErrGemmWait)) { ok = false; break; }
+          tc::tc_fence_after();
+          const uint32_t sa = base + s * SM::STAGE_BYTES;
+          const uint32_t sb = sa + SM::A_BYTES;
+          const uint64_t da = tc::sdesc_k_sw128(sa);
+          const uint64_t db = tc::sdesc_k_sw128(sb);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)     // +32 B along K inside the swizzle atom
+            tc::umma_bf16(acc, da + 2 * kk, db + 2 * kk, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+          tc::umma_commit(&empty_bar[s]);
+        }
+        if (!ok) break;
+        tc::umma_commit(&tfull_bar[b]);
+      }
+      pdl_trigger();                             // no more tensor work: the next kernel may start
+      if (!ok) {
         s_abort = 1;
-        break;
+        // release epilogue warps that wait for accumulators that will not come
+        tc::mbar_arrive(&tfull_bar[0]);
+        tc::mbar_arrive(&tfull_bar[1]);
       }
-      uint8_t* sa = sbase + s * SM::STAGE_BYTES;
-      uint8_t* sb = sa + SM::A_BYTES;
-      tc::mbar_arrive_expect_tx(&full_bar[s], SM::STAGE_BYTES);
-      if (kb < nkb0) tc::tma_load_2d(&tmA0, &full_bar[s], sa, kb * BK, a_row);
-      else tc::tma_load_2d(&tmA1, &full_bar[s], sa, (kb - nkb0) * BK, a_row);
-      tc::tma_load_2d(&tmB, &full_bar[s], sb, kb * BK, b_row);
-      ++issued;
     }
-    // drain: the copies in flight must land before the CTA may exit
-    for (int kb = (issued > STAGES ? issued - STAGES : 0); kb < issued; ++kb)
-      tc::mbar_wait(&full_bar[kb % STAGES], (kb / STAGES) & 1, g.status, kErrGemmWait);
-  } else if (warp == 1 && lane == 0) {
-    // ---------------- MMA issuer
-    constexpr uint32_t idesc = tc::idesc_bf16_f32(BM, BN);
-    bool ok = true;
-    for (int kb = 0; kb < nkb; ++kb) {
-      const int s = kb % STAGES;
-      if (!tc::mbar_wait(&full_bar[s], (kb / STAGES) & 1, g.status, kErrGemmWait)) {
-        ok = false;
-        break;
-      }
+  } else {
+    // ---------------- epilogue warps 2..5: TMEM lane quarter = warp % 4
+    const int q = warp & 3;
+    int i = 0;
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++i) {
+      const int b = i & 1;
+      const bool have = tc::mbar_wait(&tfull_bar[b], (i >> 1) & 1, g.status, kErrGemmWait);
       tc::tc_fence_after();
-      const uint32_t sa = base + s * SM::STAGE_BYTES;
-      const uint32_t sb = sa + SM::A_BYTES;
-      const uint64_t da = tc::sdesc_k_sw128(sa);
-      const uint64_t db = tc::sdesc_k_sw128(sb);
-#pragma unroll
-      for (int kk = 0; kk < BK / 16; ++kk)   // +32 B along K inside the swizzle atom
-        tc::umma_bf16(tmem, da + 2 * kk, db + 2 * kk, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
-      tc::umma_commit(&empty_bar[s]);
-    }
-    if (ok) tc::umma_commit(&accum_bar);
-    else { s_abort = 1; tc::mbar_arrive(&accum_bar); }
-  }
-  __syncwarp();
-
-  // ---------------- epilogue: thread t owns tile row t (TMEM lane t)
-  const bool have = tc::mbar_wait(&accum_bar, 0, g.status, kErrGemmWait);
-  tc::tc_fence_after();
-  const int row = m0 + threadIdx.x;
-  const bool row_ok = have && row < g.rows && !s_abort;
-  const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+      if (!have || s_abort) break;
+      const int tn = t % ntn, tm = (t / ntn) % ntm, bz = t / (ntn * ntm);
+      const int n0 = tn * BN;
+      const int row = tm * BM + q * 32 + lane;
+      const bool row_ok = row < g.rows;
+      const uint32_t trow = tmem + b * BNA + ((uint32_t)(q * 32) << 16);
 #pragma unroll 1
-  for (int c0 = 0; c0 < BN; c0 += 32) {
-    float v[32];
-    tc::tmem_ld32(trow + c0, v);        // warp-collective: every lane takes part
-    if (!row_ok || n0 + c0 >= g.cols) continue;
-    const long long obase = (long long)bz * g.strideO + (long long)row * g.ldo + n0 + c0;
-    const int ncol = min(32, g.cols - (n0 + c0));
-    if (EPI == EPI_BIAS || EPI == EPI_BIAS_RELU) {
-      __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(g.out) + obase;
-      if (ncol == 32) {
-        uint4 pk[4];
-        uint32_t* p = reinterpret_cast<uint32_t*>(pk);
+      for (int c0 = 0; c0 < BN; c0 += 32) {
+        float v[32];
+        tc::tmem_ld32(trow + c0, v);             // warp-collective: every lane takes part
+        if (!row_ok || n0 + c0 >= g.cols) continue;
+        const long long obase = (long long)bz * g.strideO + (long long)row * g.ldo + n0 + c0;
+        const int ncol = min(32, g.cols - (n0 + c0));
+        if (EPI == EPI_BIAS || EPI == EPI_BIAS_RELU) {
+          __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(g.out) + obase;
+          if (ncol == 32) {
+            uint4 pk[4];
+            uint32_t* p = reinterpret_cast<uint32_t*>(pk);
+            const float4* b4 = reinterpret_cast<const float4*>(g.bias + n0 + c0);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          float a = v[2 * i] + __ldg(g.bias + n0 + c0 + 2 * i);
-          float b = v[2 * i + 1] + __ldg(g.bias + n0 + c0 + 2 * i + 1);
-          if (EPI == EPI_BIAS_RELU) { a = fmaxf(a, 0.f); b = fmaxf(b, 0.f); }
-          p[i] = tc::pack_bf16x2(a, b);
-        }
-        uint4* o4 = reinterpret_cast<uint4*>(o);
+            for (int k = 0; k < 8; ++k) {
+              const float4 bb = __ldg(b4 + k);
+              float x0 = v[4 * k] + bb.x, x1 = v[4 * k + 1] + bb.y, x2 = v[4 * k + 2] + bb.z, x3 = v[4 * k + 3] + bb.w;
+              if (EPI == EPI_BIAS_RELU) {
+                x0 = fmaxf(x0, 0.f); x1 = fmaxf(x1, 0.f); x2 = fmaxf(x2, 0.f); x3 = fmaxf(x3, 0.f);
+              }
+              p[2 * k] = tc::pack_bf16x2(x0, x1);
+              p[2 * k + 1] = tc::pack_bf16x2(x2, x3);
+            }
+            uint4* o4 = reinterpret_cast<uint4*>(o);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) o4[i] = pk[i];
-      } else {
-        for (int i = 0; i < ncol; ++i) {
-          float a = v[i] + g.bias[n0 + c0 + i];
-          if (EPI == EPI_BIAS_RELU) a = fmaxf(a, 0.f);
-          o[i] = __float2bfloat16_rn(a);
+            for (int k = 0; k < 4; ++k) o4[k] = pk[k];
+          } else {
+            for (int k = 0; k < ncol; ++k) {
+              float x = v[k] + g.bias[n0 + c0 + k];
+              if (EPI == EPI_BIAS_RELU) x = fmaxf(x, 0.f);
+              o[k] = __float2bfloat16_rn(x);
+            }
+          }
+        } else if (EPI == EPI_RESIDUAL) {
+          float* x = reinterpret_cast<float*>(g.out) + obase;
+          __nv_bfloat16* xb = reinterpret_cast<__nv_bfloat16*>(g.out2) + obase;
+          if (ncol == 32) {
+            float4* x4 = reinterpret_cast<float4*>(x);
+            uint4 pk[4];
+            uint32_t* p = reinterpret_cast<uint32_t*>(pk);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              float4 r = x4[k];
+              r.x += v[4 * k]; r.y += v[4 * k + 1]; r.z += v[4 * k + 2]; r.w += v[4 * k + 3];
+              x4[k] = r;
+              p[2 * k] = tc::pack_bf16x2(r.x, r.y);
+              p[2 * k + 1] = tc::pack_bf16x2(r.z, r.w);
+            }
+            uint4* o4 = reinterpret_cast<uint4*>(xb);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) o4[k] = pk[k];
+          } else {
+            for (int k = 0; k < ncol; ++k) {
+              const float r = x[k] + v[k];
+              x[k] = r;
+              xb[k] = __float2bfloat16_rn(r);
+            }
+          }
+        } else {
+          float* o = reinterpret_cast<float*>(g.out) + obase;
+          if (ncol == 32 && (g.ldo % 4) == 0 && (g.strideO % 4) == 0) {
+            float4* o4 = reinterpret_cast<float4*>(o);
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+              o4[k] = make_float4(v[4 * k] * g.scale, v[4 * k + 1] * g.scale, v[4 * k + 2] * g.scale,
+                                  v[4 * k + 3] * g.scale);
+          } else {
+            for (int k = 0; k < ncol; ++k) o[k] = v[k] * g.scale;
+          }
         }
       }
-    } else if (EPI == EPI_RESIDUAL) {
-      float* x = reinterpret_cast<float*>(g.out) + obase;
-      __nv_bfloat16* xb = reinterpret_cast<__nv_bfloat16*>(g.out2) + obase;
-      if (ncol == 32) {
-        float4* x4 = reinterpret_cast<float4*>(x);
-        uint4 pk[4];
-        uint32_t* p = reinterpret_cast<uint32_t*>(pk);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          float4 r = x4[i];
-          r.x += v[4 * i]; r.y += v[4 * i + 1]; r.z += v[4 * i + 2]; r.w += v[4 * i + 3];
-          x4[i] = r;
-          p[2 * i] = tc::pack_bf16x2(r.x, r.y);
-          p[2 * i + 1] = tc::pack_bf16x2(r.z, r.w);
-        }
-        uint4* o4 = reinterpret_cast<uint4*>(xb);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) o4[i] = pk[i];
-      } else {
-        for (int i = 0; i < ncol; ++i) {
-          const float r = x[i] + v[i];
-          x[i] = r;
-          xb[i] = __float2bfloat16_rn(r);
-        }
-      }
-    } else {
-      float* o = reinterpret_cast<float*>(g.out) + obase;
-      for (int i = 0; i < ncol; ++i) o[i] = v[i] * g.scale;
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&tempty_bar[b]);
     }
   }
   tc::tc_fence_before();
   __syncthreads();
-  if (warp == 0) tc::tmem_dealloc(tmem, tmem_cols<BN>());
+  if (warp == 1) tc::tmem_dealloc(tmem, 2 * BNA);
 }
 
 // ------------------------------------------------------------------ host side
@@ -253,9 +312,19 @@ bool make_bf16_map(CUtensorMap* m, const void* ptr, long long rows, long long co
 
 namespace {
 
+int num_sms_cached() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+  }
+  return n;
+}
+
 template <int BN, int STAGES, int EPI>
 cudaError_t launch_t(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b, const TcArgs& t,
-                     dim3 grid, cudaStream_t s) {
+                     int grid, cudaStream_t s) {
   auto kern = gemm_tc_kernel<BN, STAGES, EPI>;
   constexpr int smem = Smem<BN, STAGES>::BYTES;
   static bool attr = false;
@@ -264,13 +333,22 @@ cudaError_t launch_t(const CUtensorMap& a0, const CUtensorMap& a1, const CUtenso
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  kern<<<grid, kThreads, smem, s>>>(a0, a1, b, t);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute la[1];
+  la[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // overlap with the previous kernel
+  la[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = la;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, a0, a1, b, t);
 }
 
 template <int BN, int STAGES>
 cudaError_t launch_epi(int epi, const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b,
-                       const TcArgs& t, dim3 grid, cudaStream_t s) {
+                       const TcArgs& t, int grid, cudaStream_t s) {
   switch (epi) {
     case EPI_BIAS: return launch_t<BN, STAGES, EPI_BIAS>(a0, a1, b, t, grid, s);
     case EPI_BIAS_RELU: return launch_t<BN, STAGES, EPI_BIAS_RELU>(a0, a1, b, t, grid, s);
@@ -288,14 +366,21 @@ bool tc_available() { return get_encode() != nullptr; }
 cudaError_t launch_gemm_tc(const GemmArgs& g, int epi, int batch, cudaStream_t s, unsigned* status) {
   if (g.rows <= 0 || g.cols <= 0 || batch <= 0) return cudaSuccess;
   if (g.K % BK || g.k_split % BK || g.lda % 8) return cudaErrorInvalidValue;
-  // Column tile: wide enough to amortise the A tile, narrow enough to fill the SMs.
-  int BN;
+  // Column tile: fewest waves of (tile work + a fixed per-tile latency) over the
+  // SMs; among ties the wider tile (A is read fewer times).
+  const int nsm = num_sms_cached();
   const long long row_tiles = (long long)((g.rows + BM - 1) / BM) * batch;
-  if (epi == EPI_SCALE) BN = 128;
-  else if (g.cols % 256 == 0 && row_tiles * (g.cols / 256) >= 148) BN = 256;
-  else if (g.cols % 128 == 0 && row_tiles * (g.cols / 128) >= 120) BN = 128;
-  else if (g.cols % 64 == 0) BN = 64;
-  else BN = 128;
+  int BN = 64;
+  double best = 1e300;
+  const int cands[4] = {256, 192, 128, 64};
+  for (int ci = 0; ci < 4; ++ci) {
+    const int bn = cands[ci];
+    if (bn != 64 && g.cols % bn != 0) continue;
+    const long long tiles = row_tiles * ((g.cols + bn - 1) / bn);
+    const double waves = std::ceil((double)tiles / nsm);
+    const double cost = waves * (bn + 64.0);
+    if (cost < best - 1e-9) { best = cost; BN = bn; }
+  }
   // A rows: rows of one batch item live at strideA / lda rows apart
   const long long a_batch_rows = batch > 1 ? g.strideA / g.lda : 0;
   const long long b_batch_rows = batch > 1 ? g.strideW / g.K : 0;
@@ -312,15 +397,17 @@ cudaError_t launch_gemm_tc(const GemmArgs& g, int epi, int batch, cudaStream_t s
   const long long b_total_rows = batch > 1 ? b_batch_rows * (batch - 1) + g.cols : g.cols;
   if (!make_bf16_map(&b, g.W, b_total_rows, g.K, g.K, BN)) return cudaErrorInvalidValue;
   TcArgs t{};
-  t.rows = g.rows; t.cols = g.cols; t.K = g.K; t.k_split = g.k_split;
+  t.rows = g.rows; t.cols = g.cols; t.K = g.K; t.k_split = g.k_split; t.batch = batch;
   t.a_batch_rows = (int)a_batch_rows;
   t.b_batch_rows = (int)b_batch_rows;
   t.b_row0 = 0;
   t.bias = g.bias; t.out = g.out; t.out2 = g.out2; t.ldo = g.ldo; t.strideO = g.strideO;
   t.scale = g.scale; t.status = status;
-  dim3 grid((g.cols + BN - 1) / BN, (g.rows + BM - 1) / BM, batch);
+  const long long tiles = row_tiles * ((g.cols + BN - 1) / BN);
+  const int grid = (int)(tiles < nsm ? tiles : nsm);
   switch (BN) {
     case 256: return launch_epi<256, 3>(epi, a0, a1, b, t, grid, s);
+    case 192: return launch_epi<192, 4>(epi, a0, a1, b, t, grid, s);
     case 128: return launch_epi<128, 4>(epi, a0, a1, b, t, grid, s);
     default: return launch_epi<64, 6>(epi, a0, a1, b, t, grid, s);
   }

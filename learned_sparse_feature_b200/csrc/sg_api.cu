@@ -56,6 +56,8 @@ struct sg_handle {
   // weights
   float* encW[SG_ENC_LAYERS];
   float* encb[SG_ENC_LAYERS];
+  void* encW3;         // bf16 256 x 128 (folded BN), tensor-core encoder layer 3
+  void* encW4;         // bf16 256 x 256, encoder layer 4
   std::vector<StageW> stages;
   void* Wf;
   float* bf;
@@ -175,6 +177,8 @@ sg_status_t pack_weights(sg_handle* h, const sg_weights* w) {
       for (int i = 0; i < L.in; ++i) Wt[(size_t)i * L.out + o] = L.W[(size_t)o * L.in + i];
     h->encW[l] = upload_f32(h, Wt, &ok);
     h->encb[l] = upload_f32(h, L.b, &ok);
+    if (h->bf16 && l == 3) h->encW3 = upload_matrix<__nv_bfloat16>(h, L.W, L.W.size(), &ok);
+    if (h->bf16 && l == 4) h->encW4 = upload_matrix<__nv_bfloat16>(h, L.W, L.W.size(), &ok);
   }
   const int D = kD;
   h->stages.resize(c.n_stages);
@@ -264,9 +268,30 @@ cudaError_t run_network(sg_handle* h, int B, int M, int N, const Inputs& in, flo
   const float mx = c.img_w > c.img_h ? c.img_w : c.img_h;
   ea.inv_scale = (float)(1.0 / (c.norm_mode == 0 ? 0.7 * (double)mx : 0.5 * (double)mx));
   mark(h, s, K_ENCODER);
-  cudaError_t e = launch_encoder(ea, h->bf16, s);
-  ++*launches;
-  if (e != cudaSuccess) return e;
+  cudaError_t e;
+  if (h->use_tc) {
+    // layers 0-2 on CUDA cores, layers 3-4 on the tensor cores
+    __nv_bfloat16* h2 = reinterpret_cast<__nv_bfloat16*>(h->msg);   // R x 128, free until attention
+    e = launch_encoder_head(ea, h2, s);
+    ++*launches;
+    if (e != cudaSuccess) return e;
+    GemmArgs g{};
+    g.A0 = h2; g.A1 = nullptr; g.lda = 128; g.k_split = 128;
+    g.W = h->encW3; g.bias = h->encb[3]; g.out = h->hid; g.ldo = kD;
+    g.rows = R; g.cols = kD; g.K = 128; g.scale = 1.f;
+    ++*launches;
+    if ((e = launch_gemm_tc(g, EPI_BIAS_RELU, 1, s, h->status)) != cudaSuccess) return e;
+    g = GemmArgs{};
+    g.A0 = h->hid; g.A1 = nullptr; g.lda = kD; g.k_split = kD;
+    g.W = h->encW4; g.bias = nullptr; g.out = h->x32; g.out2 = h->x16; g.ldo = kD;
+    g.rows = R; g.cols = kD; g.K = kD; g.scale = 1.f;
+    ++*launches;
+    if ((e = launch_gemm_tc(g, EPI_RESIDUAL, 1, s, h->status)) != cudaSuccess) return e;
+  } else {
+    e = launch_encoder(ea, h->bf16, s);
+    ++*launches;
+    if (e != cudaSuccess) return e;
+  }
   const void* xin = h->bf16 ? (const void*)h->x16 : (const void*)h->x32;
   for (int st = 0; st < c.n_stages; ++st) {
     const StageW& w = h->stages[st];
@@ -438,7 +463,7 @@ const char* sg_strerror(sg_status_t s) {
 
 int sg_launches_per_match(const sg_handle* h, int B, int M, int N) {
   if (!h || B == 0 || M == 0 || N == 0) return 0;
-  return 4 + 4 * h->cfg.n_stages;
+  return (h->use_tc ? 6 : 4) + 4 * h->cfg.n_stages;
 }
 
 sg_status_t sg_create(const sg_weights* w, const sg_config* cfg, sg_handle** out) {

@@ -101,6 +101,8 @@ struct SinkhornArgs {
 
 // ------------------------------------------------------------------ launchers
 cudaError_t launch_encoder(const EncArgs& a, bool write_bf16, cudaStream_t s);
+// bf16 path: layers 0-2 -> h2 (points x 128, bf16) and x32 = descriptors
+cudaError_t launch_encoder_head(const EncArgs& a, __nv_bfloat16* h2, cudaStream_t s);
 cudaError_t launch_gemm_simt(const GemmArgs& g, int epi, bool in_bf16, bool out_bf16,
                              int batch, cudaStream_t s);
 cudaError_t launch_attention_simt(const AttnArgs& a, bool bf16, cudaStream_t s);
