@@ -40,6 +40,22 @@ def shard_pairs(pairs_per_rank: int, rank: int):
     return rank * pairs_per_rank
 
 
+def reduce_max(x: float, dist=None, device=None) -> float:
+    """Max of a per-rank scalar over all ranks (the step time of a weak-scaling run
+    is the slowest rank's); identity on one process."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(x)
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(pairs_per_rank: int, world: int, steps: int, total_ms_max: float) -> float:
+    """Whole-job throughput: every rank's pairs over the slowest rank's time."""
+    return pairs_per_rank * world * steps / (total_ms_max / 1000.0)
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -273,13 +289,9 @@ def run_native(args, w):
     clk = clocks.stop()
     if world > 1:
         dist.barrier()
-    tt = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-    total_ms = float(tt.item())
+    total_ms = reduce_max(total_ms, dist if world > 1 else None, dev)
     ms_per_step = total_ms / args.steps
-    pairs = B * world * args.steps
-    value = pairs / (total_ms / 1000.0)
+    value = whole_job_rate(B, world, args.steps, total_ms)
 
     # per-kernel breakdown: same steps with events between the launches
     m.profile(True)
@@ -307,10 +319,7 @@ def run_native(args, w):
     for _ in range(max(1, args.warmup)):
         e2e_step()
     e2e_ms, _ = timed(e2e_step, args.steps)
-    te = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_ms = float(te.item())
+    e2e_ms = reduce_max(e2e_ms, dist if world > 1 else None, dev)
     h2d = sum(v.numel() * v.element_size() for v in host.values())
     d2h = sum(v.numel() * v.element_size() for v in (hm0, hm1, hs0, hs1))
 
@@ -359,7 +368,7 @@ def run_native(args, w):
         "roofline": roofline,
         "gnn_tensor_frac": (gnn_flops / gnn_s / 1e12 / peaks["bf16_tflops"]) if gnn_s > 0 else None,
         "kernels": breakdown,
-        "e2e": {"value": B * world * args.steps / (e2e_ms / 1000.0), "unit": UNIT,
+        "e2e": {"value": whole_job_rate(B, world, args.steps, e2e_ms), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "note": "sg_match_host: pinned H2D of inputs, pass, D2H of matches and scores"},
         "gpu_launches": m.launches_per_match(B, M, N) * args.steps,
