@@ -208,6 +208,17 @@ sg_status_t sg_status(sg_handle* h, void* stream);
 sg_status_t sg_selftest_barrier_timeout(sg_handle* h, unsigned timeout_us, void* stream);
 
 /*
+ * Self-test of the FMA-pipe exponential that the attention softmax uses for part
+ * of its exp2 evaluations (Cody-Waite reduction + cubic; not in the pages, which
+ * only specify the softmax).  Computes y[i] = 2^x[i] for n device floats with
+ * x clamped to [-125, 126], on `stream` (asynchronous).  x and y are device
+ * pointers owned by the caller, n >= 0 (n odd is fine).  Returns
+ * SG_ERR_INVALID_ARG on a null pointer with n > 0, SG_ERR_CUDA if the launch
+ * fails.  Expected accuracy: relative error below 1e-4 against 2^x.
+ */
+sg_status_t sg_selftest_exp2_poly(const float* x, float* y, int n, void* stream);
+
+/*
  * Per-kernel timing.  While enabled, sg_match records a CUDA event before every
  * kernel (and the Sinkhorn scratch clear) and one after the last; the events
  * are part of the captured graph.  After the stream has been synchronised,

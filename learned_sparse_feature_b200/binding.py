@@ -26,7 +26,7 @@ STATUS = {0: "SG_OK", 1: "SG_ERR_INVALID_ARG", 2: "SG_ERR_SHAPE", 3: "SG_ERR_OOM
 EXPORTED = ["sg_create", "sg_destroy", "sg_match", "sg_match_host", "sg_scores",
             "sg_optimal_transport", "sg_status", "sg_strerror", "sg_launches_per_match",
             "sg_selftest_barrier_timeout", "sg_profile", "sg_profile_read",
-            "sg_optimal_transport_static"]
+            "sg_optimal_transport_static", "sg_selftest_exp2_poly"]
 
 KERNEL_CLASSES = ["encoder", "qkv_gemm", "attention", "mlp1_gemm", "mlp2_gemm", "proj_gemm",
                   "score_gemm", "sinkhorn"]
@@ -105,6 +105,8 @@ def load():
     lib.sg_profile_read.restype = i32
     lib.sg_optimal_transport_static.argtypes = [i32, i32, i32, vp, f32, i32, f32, vp, vp, vp, vp, vp, vp, vp]
     lib.sg_optimal_transport_static.restype = i32
+    lib.sg_selftest_exp2_poly.argtypes = [vp, vp, i32, vp]
+    lib.sg_selftest_exp2_poly.restype = i32
     _lib = lib
     return lib
 
@@ -245,6 +247,14 @@ def optimal_transport_static(scores, out_logP, matches0, matches1, mscores0, msc
                                            float(match_threshold), _ptr(out_logP), _ptr(matches0),
                                            _ptr(matches1), _ptr(mscores0), _ptr(mscores1), _ptr(status),
                                            _stream_ptr(stream)), "sg_optimal_transport_static")
+
+
+def selftest_exp2_poly(x, y, stream=None):
+    """sg_selftest_exp2_poly: y = 2^x (FMA-pipe exponential of the attention
+    softmax) for float32 device tensors of equal size."""
+    lib = load()
+    n = x.numel()
+    _check(lib.sg_selftest_exp2_poly(_ptr(x), _ptr(y), int(n), _stream_ptr(stream)), "sg_selftest_exp2_poly")
 
 
 def match_batch(matcher: Matcher, batch: dict, with_logP: bool = True, stream=None):

@@ -8,24 +8,27 @@
 //
 // One CTA = one 128-query tile of one (pair, image, head); it walks the source
 // image in 128-key tiles j = 0, 1, ...:
-//   warp 8 (one lane)  TMA: Q once, then K and V tiles into a 4-deep ring;
-//   warp 9 (one lane)  MMA: S_j = Q K_j^T (M=128, N=128, K=64) into TMEM score
-//                      buffer j%2, then O_{j%2} += P_j V_j (M=128, N=64, K=128, V read
-//                      MN-major) into TMEM output buffer j%2;
+//   warp 8 (one lane)  TMA: Q once, then K and V tiles into a 6-deep ring;
+//   warp 9 (one lane)  MMA: S_j = Q K_j^T (M=128, N=128, K=64) into TMEM buffer
+//                      j%3, then O_{j%2} += P_j V_j (M=128, N=64, K=128) with P_j
+//                      read from TMEM (it overwrites S_j in its buffer) and V_j
+//                      from shared memory (MN-major); S_{j+3} is issued right
+//                      after P_j V_j, which the in-order tensor pipe finishes first;
 //   warps 0-3, 4-7     two softmax warpgroups; group g takes the tiles j = g mod 2,
 //                      thread t = query row t = TMEM lane t.  Each group keeps its own
-//                      running max and sum for its half of the keys and its own
+//                      reference max and sum for its half of the keys and its own
 //                      output accumulator in TMEM; the two halves are merged at the
 //                      end (the softmax normaliser is a sum over keys, so it splits).
-// Softmax of a tile: the 128 scores come out of TMEM, exp2 on the MUFU, P_j goes to
-// shared memory as bf16 in the 128-byte-swizzled K-major layout the MMA reads.  The
-// reference max of a row only moves when a tile's max exceeds it by more than 2^8
-// (P stays <= 256, exact in fp32 and bf16 range); then that group's TMEM output
-// row is rescaled in place before the next P V accumulates into it.
-// S_{j+2} is issued before P_j V_j, so a group finds its next scores ready when it
-// finishes a tile.  Every wait is bounded.  Launched with programmatic dependent
-// launch (prologue overlaps the previous kernel; griddepcontrol.wait gates the
-// first read of q|k|v).
+// Softmax of a tile: the 128 scores come out of TMEM, p = 2^(s log2e/8 - m) in
+// fp32 is packed to bf16 pairs and stored back into the first 64 columns of the
+// same TMEM buffer for the P V product.  The reference max m of a row is its first
+// tile's max; later tiles reuse it as long as their sum of p stays below 2^64
+// (then p <= 2^64: no overflow in fp32, bf16 or the fp32 accumulators); a tile
+// that exceeds that renews m, recomputes its p and rescales the group's TMEM
+// output row.  With three score buffers a group never waits for its own previous
+// P V before writing the next P.  Every wait is bounded.  Launched with
+// programmatic dependent launch (prologue overlaps the previous kernel;
+// griddepcontrol.wait gates the first read of q|k|v).
 #include "sg_internal.cuh"
 #include "tc_common.cuh"
 
@@ -40,28 +43,29 @@ namespace {
 
 constexpr int QT = 128;      // queries per CTA
 constexpr int KT = 128;      // keys per tile
-constexpr int ST = 4;        // K/V ring depth
+constexpr int ST = 6;        // K/V ring depth
+constexpr int NSB = 3;       // TMEM score / P buffers
 constexpr int kSoftmaxThreads = 256;
 constexpr int kThreads = kSoftmaxThreads + 64;
 constexpr unsigned kErr = 4u;
-constexpr float kRescaleLog2 = 8.f;   // lazy rescale threshold (P <= 2^8)
 
 constexpr int Q_BYTES = QT * kDh * 2;           // 16 KB
 constexpr int KV_TILE = KT * kDh * 2;           // 16 KB
 constexpr int STAGE_BYTES = 2 * KV_TILE;        // K + V
-constexpr int P_BYTES = QT * KT * 2;            // 32 KB (two 64-key swizzled sub-tiles)
 constexpr int OFF_KV = Q_BYTES;
-constexpr int OFF_P = OFF_KV + ST * STAGE_BYTES;
-constexpr int SMEM_BYTES = OFF_P + 2 * P_BYTES + 1024;
+constexpr int SMEM_BYTES = OFF_KV + ST * STAGE_BYTES + 1024;
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 
-// TMEM columns: S buffers [0,128) and [128,256); O accumulators [256,320), [320,384)
-constexpr uint32_t TM_S0 = 0, TM_O0 = 256, TMEM_COLS = 512;
+// TMEM columns: score / P buffers [0,128), [128,256), [256,384); O accumulators
+// [384,448) and [448,512)
+constexpr uint32_t TM_S0 = 0, TM_O0 = NSB * KT, TMEM_COLS = 512;
+static_assert(TM_O0 + 2 * kDh <= TMEM_COLS, "tensor memory");
 
 struct AttnTcArgs {
   __nv_bfloat16* msg;
   int B, M, N, cross;
   float scale_log2;
+  float blind_limit;
   unsigned* status;
 };
 
@@ -74,9 +78,6 @@ __device__ __forceinline__ float fast_ex2(float x) {
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
 
 __device__ __forceinline__ void softmax_bar() {
   asm volatile("bar.sync 1, %0;" ::"n"(kSoftmaxThreads) : "memory");
@@ -89,12 +90,64 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, unsign
   return __all_sync(0xffffffffu, ok);
 }
 
+// Largest of a row's 128 raw scores (four independent chains).
+__device__ __forceinline__ float row_max(const float (&s)[KT]) {
+  float t0 = -INFINITY, t1 = -INFINITY, t2 = -INFINITY, t3 = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < KT; i += 8) {
+    t0 = tc::max3(t0, s[i], s[i + 1]);
+    t1 = tc::max3(t1, s[i + 2], s[i + 3]);
+    t2 = tc::max3(t2, s[i + 4], s[i + 5]);
+    t3 = tc::max3(t3, s[i + 6], s[i + 7]);
+  }
+  return fmaxf(fmaxf(t0, t1), fmaxf(t2, t3));
+}
+
+// p = 2^(s * scale - m) for the row's 128 scores, packed to bf16 pairs and stored
+// into TMEM columns [tp, tp + 64) of this thread's lane; returns the fp32 sum.
+// EMU of every 8 pairs take the FMA-pipe exponential, the rest the MUFU.
+template <int EMU>
+__device__ __forceinline__ float exp_row(const float (&s)[KT], float scale, float m, uint32_t tp) {
+  const uint64_t sc2 = tc::f2(scale, scale);
+  const uint64_t nm2 = tc::f2(-m, -m);
+  uint64_t sa = tc::f2(0.f, 0.f), sb = sa;
+#pragma unroll
+  for (int cc = 0; cc < KT / 16; ++cc) {
+    uint32_t pk[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int i = cc * 16 + 2 * e;
+      const uint64_t x2 = tc::f2_fma(tc::f2(s[i], s[i + 1]), sc2, nm2);
+      uint64_t p2;
+      if (((cc * 8 + e) & 7) < EMU) {
+        p2 = tc::f2_exp2_poly(x2);
+      } else {
+        float x0, x1;
+        tc::f2_split(x2, x0, x1);
+        p2 = tc::f2(fast_ex2(x0), fast_ex2(x1));
+      }
+      if (e & 1) sb = tc::f2_add(sb, p2); else sa = tc::f2_add(sa, p2);
+      float p0, p1;
+      tc::f2_split(p2, p0, p1);
+      pk[e] = tc::pack_bf16x2(p0, p1);
+    }
+    tc::tmem_st8(tp + cc * 8, pk);
+  }
+  float a0, a1, b0, b1;
+  tc::f2_split(sa, a0, a1);
+  tc::f2_split(sb, b0, b1);
+  return (a0 + a1) + (b0 + b1);
+}
+
+template <int EMU>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tm, AttnTcArgs a) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t q_full;
   __shared__ __align__(8) uint64_t kv_full[ST], kv_empty[ST];
-  __shared__ __align__(8) uint64_t s_full[2], s_empty[2], p_full[2], o_full[2];
+  __shared__ __align__(8) uint64_t s_full[NSB], p_full[NSB];
+  // o_full[g][i & 1] completes when the i-th P V of group g has landed
+  __shared__ __align__(8) uint64_t o_full[2][2];
   __shared__ float2 part_ml[2][QT];      // per group and row: (reference max, sum)
   __shared__ uint32_t tmem_slot;
   __shared__ int s_abort;
@@ -120,12 +173,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm, AttnTcArgs a) {
   if (threadIdx.x == 0) {
     tc::mbar_init(&q_full, 1);
     for (int s = 0; s < ST; ++s) { tc::mbar_init(&kv_full[s], 1); tc::mbar_init(&kv_empty[s], 1); }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < NSB; ++b) {
       tc::mbar_init(&s_full[b], 1);
-      tc::mbar_init(&s_empty[b], 4);
       tc::mbar_init(&p_full[b], 4);
-      tc::mbar_init(&o_full[b], 1);
     }
+    for (int b = 0; b < 4; ++b) tc::mbar_init(&o_full[b >> 1][b & 1], 1);
     tc::fence_barrier_init();
     s_abort = 0;
   }
@@ -165,10 +217,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm, AttnTcArgs a) {
       const uint64_t dq = tc::sdesc_k_sw128(base);
       bool ok = tc::mbar_wait(&q_full, 0, a.status, kErr);
       auto issue_s = [&](int j) -> bool {
-        const int st = j % ST, b = j & 1;
+        const int st = j % ST, b = j % NSB;
         if (!tc::mbar_wait(&kv_full[st], (j / ST) & 1, a.status, kErr)) return false;
-        if (j >= 2 && !tc::mbar_wait(&s_empty[b], ((j >> 1) - 1) & 1, a.status, kErr)) return false;
         tc::tc_fence_after();
+        // buffer b last held P_{j-3}; P_{j-3} V_{j-3} was issued before this and
+        // the tensor pipe runs this thread's MMAs in order
         const uint64_t dk = tc::sdesc_k_sw128(base + OFF_KV + st * STAGE_BYTES);
 #pragma unroll
         for (int kk = 0; kk < kDh / 16; ++kk)
@@ -177,25 +230,25 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm, AttnTcArgs a) {
         return true;
       };
       auto issue_pv = [&](int j) -> bool {
-        const int b = j & 1;
-        if (!tc::mbar_wait(&p_full[b], (j >> 1) & 1, a.status, kErr)) return false;
+        const int b = j % NSB;
+        if (!tc::mbar_wait(&p_full[b], (j / NSB) & 1, a.status, kErr)) return false;
         tc::tc_fence_after();
-        const uint32_t pbase = base + OFF_P + b * P_BYTES;
         const uint32_t vbase = base + OFF_KV + (j % ST) * STAGE_BYTES + KV_TILE;
 #pragma unroll
         for (int kk = 0; kk < KT / 16; ++kk) {
-          const uint64_t da = tc::sdesc_k_sw128(pbase + (kk >> 2) * (QT * 128)) + 2 * (kk & 3);
           const uint64_t dv = tc::sdesc_mn_sw128(vbase + kk * 2048, 8192, 1024);
-          tc::umma_bf16(tmem + TM_O0 + b * kDh, da, dv, idesc_o, (j >= 2 || kk > 0) ? 1u : 0u);
+          // 16 keys of P = 8 TMEM columns of bf16 pairs
+          tc::umma_bf16_ts(tmem + TM_O0 + (j & 1) * kDh, tmem + TM_S0 + b * KT + kk * 8, dv, idesc_o,
+                           (j >= 2 || kk > 0) ? 1u : 0u);
         }
-        tc::umma_commit(&o_full[b]);
+        tc::umma_commit(&o_full[j & 1][(j >> 1) & 1]);
         tc::umma_commit(&kv_empty[j % ST]);
         return true;
       };
-      for (int j = 0; ok && j < 2 && j < ntiles; ++j) ok = issue_s(j);
+      for (int j = 0; ok && j < NSB && j < ntiles; ++j) ok = issue_s(j);
       for (int j = 0; ok && j < ntiles; ++j) {
-        if (j + 2 < ntiles) ok = issue_s(j + 2);
-        if (ok) ok = issue_pv(j);
+        ok = issue_pv(j);
+        if (ok && j + NSB < ntiles) ok = issue_s(j + NSB);
       }
       pdl_trigger();                             // no more tensor work: the next kernel may start
       if (!ok) s_abort = 1;
@@ -205,14 +258,24 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm, AttnTcArgs a) {
     const int g = warp >> 2;
     const int r = threadIdx.x & (QT - 1);            // query row = TMEM lane
     const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-    const uint32_t t_s = tl + TM_S0 + g * KT;
     const uint32_t t_o = tl + TM_O0 + g * kDh;
-    uint8_t* prow = sb + OFF_P + g * P_BYTES + (r >> 3) * 1024 + (r & 7) * 128;
     float m = -INFINITY, l = 0.f;                    // log2-domain reference max, running sum
     int k = 0;                                       // tiles this group has taken
+    int pv_seen = 0;                                 // completions of o_full[g] waited for
     bool ok = true;
+    // wait, in order, for this group's P V products up to count `upto`.  P V
+    // number i completes on o_full[g][i & 1]; a group waits for number i only
+    // after it has issued at most i + 2 of them, so neither barrier can be two
+    // phases ahead of the parity asked for
+    auto wait_pv = [&](int upto) -> bool {
+      for (; pv_seen < upto; ++pv_seen)
+        if (!warp_wait(&o_full[g][pv_seen & 1], (pv_seen >> 1) & 1, a.status)) return false;
+      return true;
+    };
     for (int j = g; j < ntiles; j += 2, ++k) {
-      if (!warp_wait(&s_full[g], k & 1, a.status)) { ok = false; break; }
+      const int b = j % NSB;
+      const uint32_t t_s = tl + TM_S0 + b * KT;
+      if (!warp_wait(&s_full[b], (j / NSB) & 1, a.status)) { ok = false; break; }
       tc::tc_fence_after();
       float s[KT];
       {
@@ -226,60 +289,35 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm, AttnTcArgs a) {
         tc::tmem_ld32_async(t_s + 96, s3);
         tc::tmem_wait_ld();
       }
-      tc::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&s_empty[g]);
       const int valid = nk - j * KT;                 // keys of this tile that exist
       if (valid < KT) {
 #pragma unroll
         for (int i = 0; i < KT; ++i)
           if (i >= valid) s[i] = -INFINITY;
       }
-      float t0 = s[0], t1 = s[1];
-#pragma unroll
-      for (int i = 2; i < KT; i += 4) {
-        t0 = tc::max3(t0, s[i], s[i + 1]);
-        t1 = tc::max3(t1, s[i + 2], s[i + 3]);
-      }
-      const float tmax = fmaxf(t0, t1) * a.scale_log2;
-      const bool need = tmax > m + kRescaleLog2;
-      // the previous P_{j-2} V_{j-2} must be done: it reads the P buffer about to
-      // be overwritten and accumulates into the output row that may be rescaled
-      if (k >= 1 && !warp_wait(&o_full[g], (k - 1) & 1, a.status)) { ok = false; break; }
+      // reference max of the row: the first tile's max; later tiles reuse it
+      // unless their exponentials overflow the budget checked below
+      if (k == 0) m = row_max(s) * a.scale_log2;
+      // consume the completion of this group's P V two tiles back (long done)
+      if (!wait_pv(k - 1)) { ok = false; break; }
+      float sum = exp_row<EMU>(s, a.scale_log2, m, t_s);
+      const bool redo = !(sum <= a.blind_limit);     // a score far above m (or a NaN)
       float c = 1.f;
-      if (need) {
-        c = fast_ex2(m - tmax);                      // 0 on the first tile (m = -inf)
-        l *= c;
-        m = tmax;
-      }
-      const uint64_t sc2 = tc::f2(a.scale_log2, a.scale_log2);
-      const uint64_t nm2 = tc::f2(-m, -m);
-      uint64_t sum2 = tc::f2(0.f, 0.f);
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-#pragma unroll
-        for (int cc = 0; cc < 8; ++cc) {
-          uint32_t pk[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int i = half * 64 + cc * 8 + 2 * e;
-            float x0, x1;
-            tc::f2_split(tc::f2_fma(tc::f2(s[i], s[i + 1]), sc2, nm2), x0, x1);
-            const float p0 = fast_ex2(x0), p1 = fast_ex2(x1);
-            const uint64_t p2 = tc::f2(p0, p1);
-            sum2 = tc::f2_add(sum2, p2);
-            pk[e] = tc::pack_bf16x2(p0, p1);
-          }
-          *reinterpret_cast<uint4*>(prow + half * (QT * 128) + ((cc ^ (r & 7)) << 4)) =
-              make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      const bool any_redo = __any_sync(0xffffffffu, redo);
+      if (any_redo) {                                // warp-uniform: the TMEM stores need all lanes
+        if (redo) {
+          const float tmax = fmaxf(m, row_max(s) * a.scale_log2);
+          c = fast_ex2(m - tmax);
+          l *= c;
+          m = tmax;
         }
+        sum = exp_row<0>(s, a.scale_log2, m, t_s);   // (other lanes rewrite their row unchanged)
       }
-      float sa, sb2;
-      tc::f2_split(sum2, sa, sb2);
-      l += sa + sb2;
-      // (after the P writes: the 128 scores are dead and their registers free)
-      const bool rescale_o = k >= 1 && __any_sync(0xffffffffu, need);
-      if (rescale_o) {
+      l += sum;
+      // (the 128 scores are dead here and their registers free)
+      if (k >= 1 && any_redo) {
+        // every earlier P V of this group must have landed before its rows scale
+        if (!wait_pv(k)) { ok = false; break; }
         tc::tc_fence_after();
         float o[32];
 #pragma unroll
@@ -289,15 +327,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm, AttnTcArgs a) {
           for (int d = 0; d < 32; ++d) o[d] *= c;
           tc::tmem_st32(t_o + hh * 32, o);
         }
-        tc::tmem_wait_st();
       }
-      fence_proxy_async_smem();
-      if (rescale_o) tc::tc_fence_before();
+      tc::tmem_wait_st();
+      tc::tc_fence_before();
       __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&p_full[g]);
+      if (lane == 0) tc::mbar_arrive(&p_full[b]);
     }
-    // the last P V of this group must be done before its accumulator is read
-    if (ok && k >= 1 && !warp_wait(&o_full[g], (k - 1) & 1, a.status)) ok = false;
+    // every P V of this group must be done before its accumulator is read
+    if (ok && !wait_pv(k)) ok = false;
     if (!ok) s_abort = 1;
     part_ml[g][r] = make_float2(m, l);
     tc::tc_fence_before();
@@ -339,6 +376,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm, AttnTcArgs a) {
   if (warp == 9) tc::tmem_dealloc(tmem, TMEM_COLS);
 }
 
+__global__ void exp2_poly_selftest_kernel(const float* x, float* y, int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i >= n) return;
+  const float x0 = x[i], x1 = i + 1 < n ? x[i + 1] : 0.f;
+  float y0, y1;
+  tc::f2_split(tc::f2_exp2_poly(tc::f2(x0, x1)), y0, y1);
+  y[i] = y0;
+  if (i + 1 < n) y[i + 1] = y1;
+}
+
 }  // namespace
 
 cudaError_t launch_attention_tc(const AttnArgs& a, cudaStream_t s, unsigned* status) {
@@ -347,13 +394,19 @@ cudaError_t launch_attention_tc(const AttnArgs& a, cudaStream_t s, unsigned* sta
   const long long R = (long long)a.B * (a.M + a.N);
   CUtensorMap tm;
   if (!make_bf16_map(&tm, a.qkv, R, kQKV, kQKV, 128)) return cudaErrorInvalidValue;
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+  // share of the exponentials taken on the FMA pipe: exp_emu of every 8 pairs
+  const int emu = (a.exp_emu == 0 || a.exp_emu == 2 || a.exp_emu == 4) ? a.exp_emu : 3;
+  using Kern = void (*)(const CUtensorMap, AttnTcArgs);
+  Kern kern = emu == 0 ? attn_tc_kernel<0> : emu == 2 ? attn_tc_kernel<2> : emu == 4 ? attn_tc_kernel<4>
+                                                                                 : attn_tc_kernel<3>;
+  static bool attr[5] = {};
+  if (!attr[emu]) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    attr = true;
+    attr[emu] = true;
   }
-  AttnTcArgs t{reinterpret_cast<__nv_bfloat16*>(a.msg), a.B, a.M, a.N, a.cross, a.scale_log2, status};
+  AttnTcArgs t{reinterpret_cast<__nv_bfloat16*>(a.msg), a.B, a.M, a.N, a.cross, a.scale_log2,
+               a.blind_limit > 0.f ? a.blind_limit : 18446744073709551616.f, status};
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((nmax + QT - 1) / QT, kH, 2 * a.B);
   cfg.blockDim = dim3(kThreads);
@@ -364,7 +417,14 @@ cudaError_t launch_attention_tc(const AttnArgs& a, cudaStream_t s, unsigned* sta
   la[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = la;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, attn_tc_kernel, tm, t);
+  return cudaLaunchKernelEx(&cfg, kern, tm, t);
+}
+
+cudaError_t launch_exp2_poly_selftest(const float* x, float* y, int n, cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  const int pairs = (n + 1) / 2;
+  exp2_poly_selftest_kernel<<<(pairs + 255) / 256, 256, 0, s>>>(x, y, n);
+  return cudaGetLastError();
 }
 
 }  // namespace sg

@@ -61,6 +61,21 @@ template <int BN> __host__ __device__ constexpr uint32_t tmem_cols() {
   return BN <= 32 ? 32 : BN <= 64 ? 64 : BN <= 128 ? 128 : 256;
 }
 
+// Barrier of the 128 epilogue threads (named barrier 1) that also returns the
+// AND of their predicates.
+__device__ __forceinline__ bool epi_all(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, 1, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v)
+      : "memory");
+  return r != 0;
+}
+
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
@@ -80,6 +95,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
   __shared__ __align__(8) uint64_t empty_bar[STAGES];
   __shared__ __align__(8) uint64_t tfull_bar[2];
   __shared__ __align__(8) uint64_t tempty_bar[2];
+  __shared__ __align__(16) float s_bias[2][BN];   // bias of the tile, by accumulator buffer
   __shared__ uint32_t tmem_slot;
   __shared__ int s_abort;
 
@@ -185,34 +201,62 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
     }
   } else {
     // ---------------- epilogue warps 2..5: TMEM lane quarter = warp % 4
+    // While the MMA warp accumulates a tile, these warps stage its bias in
+    // shared memory and start the loads of its first residual chunk, so that no
+    // global-memory latency sits between the accumulator and the stores.
     const int q = warp & 3;
+    const int et = threadIdx.x - 64;             // 0..127
     int i = 0;
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++i) {
       const int b = i & 1;
-      const bool have = tc::mbar_wait(&tfull_bar[b], (i >> 1) & 1, g.status, kErrGemmWait);
-      tc::tc_fence_after();
-      if (!have || s_abort) break;
       const int tn = t % ntn, tm = (t / ntn) % ntm, bz = t / (ntn * ntm);
       const int n0 = tn * BN;
       const int row = tm * BM + q * 32 + lane;
       const bool row_ok = row < g.rows;
+      const long long rbase = (long long)bz * g.strideO + (long long)row * g.ldo + n0;
+      if (EPI == EPI_BIAS || EPI == EPI_BIAS_RELU) {
+        for (int c = et; c < BN; c += 128) s_bias[b][c] = (n0 + c < g.cols) ? __ldg(g.bias + n0 + c) : 0.f;
+      }
+      float4 rnext[8];
+      const bool vec_res = EPI == EPI_RESIDUAL && n0 + BN <= g.cols;   // full-width tile: float4 path
+      if (EPI == EPI_RESIDUAL && vec_res && row_ok) {
+        const float4* x4 = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(g.out) + rbase);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) rnext[k] = __ldcg(x4 + k);
+      }
+      const bool got = tc::mbar_wait(&tfull_bar[b], (i >> 1) & 1, g.status, kErrGemmWait);
+      // one barrier of the 128 epilogue threads per tile: publishes the staged
+      // bias and makes the go / stop decision the same for all of them
+      if (!epi_all(got && !s_abort)) break;
+      tc::tc_fence_after();
       const uint32_t trow = tmem + b * BNA + ((uint32_t)(q * 32) << 16);
 #pragma unroll 1
       for (int c0 = 0; c0 < BN; c0 += 32) {
         float v[32];
         tc::tmem_ld32(trow + c0, v);             // warp-collective: every lane takes part
+        float4 rcur[8];
+        if (EPI == EPI_RESIDUAL && vec_res) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) rcur[k] = rnext[k];
+          if (c0 + 32 < BN && row_ok) {
+            const float4* x4 = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(g.out) + rbase + c0 + 32);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) rnext[k] = __ldcg(x4 + k);
+          }
+        }
         if (!row_ok || n0 + c0 >= g.cols) continue;
-        const long long obase = (long long)bz * g.strideO + (long long)row * g.ldo + n0 + c0;
+        const long long obase = rbase + c0;
         const int ncol = min(32, g.cols - (n0 + c0));
         if (EPI == EPI_BIAS || EPI == EPI_BIAS_RELU) {
           __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(g.out) + obase;
+          const float* sbv = s_bias[b] + c0;
           if (ncol == 32) {
             uint4 pk[4];
             uint32_t* p = reinterpret_cast<uint32_t*>(pk);
-            const float4* b4 = reinterpret_cast<const float4*>(g.bias + n0 + c0);
+            const float4* b4 = reinterpret_cast<const float4*>(sbv);
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
-              const float4 bb = __ldg(b4 + k);
+              const float4 bb = b4[k];
               float x0 = v[4 * k] + bb.x, x1 = v[4 * k + 1] + bb.y, x2 = v[4 * k + 2] + bb.z, x3 = v[4 * k + 3] + bb.w;
               if (EPI == EPI_BIAS_RELU) {
                 x0 = fmaxf(x0, 0.f); x1 = fmaxf(x1, 0.f); x2 = fmaxf(x2, 0.f); x3 = fmaxf(x3, 0.f);
@@ -224,22 +268,25 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
 #pragma unroll
             for (int k = 0; k < 4; ++k) o4[k] = pk[k];
           } else {
-            for (int k = 0; k < ncol; ++k) {
-              float x = v[k] + g.bias[n0 + c0 + k];
-              if (EPI == EPI_BIAS_RELU) x = fmaxf(x, 0.f);
-              o[k] = __float2bfloat16_rn(x);
+#pragma unroll
+            for (int k = 0; k < 32; ++k) {           // static indices keep v in registers
+              if (k < ncol) {
+                float x = v[k] + sbv[k];
+                if (EPI == EPI_BIAS_RELU) x = fmaxf(x, 0.f);
+                o[k] = __float2bfloat16_rn(x);
+              }
             }
           }
         } else if (EPI == EPI_RESIDUAL) {
           float* x = reinterpret_cast<float*>(g.out) + obase;
           __nv_bfloat16* xb = reinterpret_cast<__nv_bfloat16*>(g.out2) + obase;
-          if (ncol == 32) {
+          if (vec_res) {
             float4* x4 = reinterpret_cast<float4*>(x);
             uint4 pk[4];
             uint32_t* p = reinterpret_cast<uint32_t*>(pk);
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
-              float4 r = x4[k];
+              float4 r = rcur[k];
               r.x += v[4 * k]; r.y += v[4 * k + 1]; r.z += v[4 * k + 2]; r.w += v[4 * k + 3];
               x4[k] = r;
               p[2 * k] = tc::pack_bf16x2(r.x, r.y);
@@ -249,10 +296,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
 #pragma unroll
             for (int k = 0; k < 4; ++k) o4[k] = pk[k];
           } else {
-            for (int k = 0; k < ncol; ++k) {
-              const float r = x[k] + v[k];
-              x[k] = r;
-              xb[k] = __float2bfloat16_rn(r);
+#pragma unroll
+            for (int k = 0; k < 32; ++k) {
+              if (k < ncol) {
+                const float r = x[k] + v[k];
+                x[k] = r;
+                xb[k] = __float2bfloat16_rn(r);
+              }
             }
           }
         } else {
@@ -264,7 +314,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
               o4[k] = make_float4(v[4 * k] * g.scale, v[4 * k + 1] * g.scale, v[4 * k + 2] * g.scale,
                                   v[4 * k + 3] * g.scale);
           } else {
-            for (int k = 0; k < ncol; ++k) o[k] = v[k] * g.scale;
+#pragma unroll
+            for (int k = 0; k < 32; ++k)
+              if (k < ncol) o[k] = v[k] * g.scale;
           }
         }
       }

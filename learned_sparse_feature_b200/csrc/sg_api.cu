@@ -53,6 +53,8 @@ struct sg_handle {
   bool bf16;
   bool use_tc;        // tcgen05 GEMMs
   bool use_tc_attn;   // tcgen05 attention
+  int attn_exp_emu;   // softmax exponentials on the FMA pipe, of every 8 pairs
+  float attn_blind_limit;   // bound on a key tile's sum of P under a stale row max
   // weights
   float* encW[SG_ENC_LAYERS];
   float* encb[SG_ENC_LAYERS];
@@ -305,6 +307,8 @@ cudaError_t run_network(sg_handle* h, int B, int M, int N, const Inputs& in, flo
     aa.qkv = h->qkv; aa.msg = h->msg; aa.B = B; aa.M = M; aa.N = N;
     aa.cross = (st % 2 == 1);
     aa.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)kDh));
+    aa.exp_emu = h->attn_exp_emu;
+    aa.blind_limit = h->attn_blind_limit;
     mark(h, s, K_ATTN);
     ++*launches;
     e = h->use_tc_attn ? launch_attention_tc(aa, s, h->status) : launch_attention_simt(aa, h->bf16, s);
@@ -490,6 +494,17 @@ sg_status_t sg_create(const sg_weights* w, const sg_config* cfg, sg_handle** out
   h->bf16 = cfg->precision == SG_PRECISION_BF16;
   h->use_tc = h->bf16 && tc_available() && std::getenv("SG_FORCE_SIMT") == nullptr;
   h->use_tc_attn = h->use_tc && std::getenv("SG_SIMT_ATTENTION") == nullptr;
+  {
+    // SG_ATTN_EXP_EMU=0|2|3|4 overrides the default share (3 of 8); for tests
+    const char* e = std::getenv("SG_ATTN_EXP_EMU");
+    const int v = e ? std::atoi(e) : 3;
+    h->attn_exp_emu = (v == 0 || v == 2 || v == 4) ? v : 3;
+    // SG_ATTN_BLIND_LIMIT_LOG2=x (0 <= x <= 64) lowers the 2^64 bound so that
+    // the max-renewal path runs on ordinary inputs; for tests
+    const char* b = std::getenv("SG_ATTN_BLIND_LIMIT_LOG2");
+    const double lb = b ? std::atof(b) : 64.0;
+    h->attn_blind_limit = (float)std::exp2(lb >= 0.0 && lb <= 64.0 ? lb : 64.0);
+  }
   h->use_graph = std::getenv("SG_NO_GRAPH") == nullptr;
   h->sticky = SG_OK;
   sg_status_t st = pack_weights(h, w);
@@ -641,6 +656,13 @@ sg_status_t sg_match_host(sg_handle* h, int B, int M, int N, const float* kpts0,
     e = d2h(out_logP, h->s_logP, (size_t)B * (M + 1) * (N + 1) * 4);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   return cuda_err(h, e);
+}
+
+sg_status_t sg_selftest_exp2_poly(const float* x, float* y, int n, void* stream) {
+  if (n < 0) return SG_ERR_INVALID_ARG;
+  if (n == 0) return SG_OK;
+  if (!x || !y) return SG_ERR_INVALID_ARG;
+  return launch_exp2_poly_selftest(x, y, n, (cudaStream_t)stream) == cudaSuccess ? SG_OK : SG_ERR_CUDA;
 }
 
 sg_status_t sg_selftest_barrier_timeout(sg_handle* h, unsigned timeout_us, void* stream) {

@@ -55,6 +55,8 @@ struct AttnArgs {
   int B, M, N;
   int cross;
   float scale_log2;   // log2(e) / sqrt(d_head)
+  int exp_emu;        // tensor-core path: of every 8 exp2 pairs, how many use the FMA pipe (0, 2, 3 or 4)
+  float blind_limit;  // tensor-core path: bound on a key tile's sum of 2^(s - m) before the row's max is renewed
 };
 
 struct EncArgs {
@@ -111,6 +113,7 @@ cudaError_t sinkhorn_prepare(int num_sms);   // kernel attributes (called once, 
 int sinkhorn_max_columns();                  // largest N the transport kernel supports
 size_t sinkhorn_scratch_bytes(int B, int M, int N);
 size_t sinkhorn_acc_floats_per_buffer(int N);   // column accumulator floats per (pair, rotation)
+cudaError_t launch_exp2_poly_selftest(const float* x, float* y, int n, cudaStream_t s);
 cudaError_t launch_barrier_selftest(unsigned* scratch, unsigned* status, unsigned long long timeout_ns,
                                     int* returned, cudaStream_t s);
 

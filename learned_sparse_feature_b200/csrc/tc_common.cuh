@@ -129,6 +129,18 @@ __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint
       : "memory");
 }
 
+// D[tmem] (+)= A[tmem] * B[smem]^T: the A operand (M rows = TMEM lanes, K along
+// columns, two bf16 per 32-bit column) is read from tensor memory.
+__device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrive on `bar` once every tcgen05.mma issued so far by this thread is done.
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
@@ -170,6 +182,17 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// 16 consecutive fp32 columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]), "=f"(v[6]), "=f"(v[7]),
+        "=f"(v[8]), "=f"(v[9]), "=f"(v[10]), "=f"(v[11]), "=f"(v[12]), "=f"(v[13]), "=f"(v[14]), "=f"(v[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
 // The same load without the wait: several loads may be in flight before one
 // tmem_wait_ld(); the registers must not be read before that wait.
 __device__ __forceinline__ void tmem_ld32_async(uint32_t taddr, float (&v)[32]) {
@@ -199,6 +222,13 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) 
         "f"(v[24]), "f"(v[25]), "f"(v[26]), "f"(v[27]), "f"(v[28]), "f"(v[29]), "f"(v[30]), "f"(v[31])
       : "memory");
 }
+// 8 consecutive 32-bit columns of this thread's TMEM lane, stored.
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&v)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"
+               ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]),
+               "r"(v[7])
+               : "memory");
+}
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // Paired fp32 arithmetic (one instruction for two lanes of a 64-bit register pair).
@@ -224,6 +254,33 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
   return r;
+}
+
+// 2^x on the FMA pipe for a pair of lanes (Cody-Waite range reduction followed by
+// a polynomial): x is clamped to [-125, 126], n = round(x) by the 1.5 * 2^23
+// addition trick, f = x - n in [-1/2, 1/2], 2^f by a cubic whose coefficients
+// are a relative-error-weighted least-squares fit on [-1/2, 1/2] (max relative
+// error 7.6e-5), and 2^n enters by an integer add to the exponent field.  Used
+// for part of the softmax exponentials so that they do not all queue on the MUFU.
+__device__ __forceinline__ uint64_t f2_exp2_poly(uint64_t x2) {
+  float x0, x1;
+  f2_split(x2, x0, x1);
+  x0 = fminf(fmaxf(x0, -125.f), 126.f);
+  x1 = fminf(fmaxf(x1, -125.f), 126.f);
+  const uint64_t xc = f2(x0, x1);
+  const uint64_t magic = f2(12582912.f, 12582912.f);                 // 1.5 * 2^23
+  const uint64_t t = f2_add(xc, magic);                              // low bits hold round(x)
+  const uint64_t n = f2_add(t, f2(-12582912.f, -12582912.f));
+  const uint64_t fr = f2_fma(n, f2(-1.f, -1.f), xc);                // x - n, exact
+  uint64_t p = f2_fma(fr, f2(0.0551863760f, 0.0551863760f), f2(0.242612362f, 0.242612362f));
+  p = f2_fma(p, fr, f2(0.693258286f, 0.693258286f));
+  p = f2_fma(p, fr, f2(0.999927938f, 0.999927938f));
+  float p0, p1, t0, t1;
+  f2_split(p, p0, p1);
+  f2_split(t, t0, t1);
+  const float r0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
+  const float r1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
+  return f2(r0, r1);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -20,7 +20,7 @@ def lib():
 def _declared():
     text = open(os.path.join(ROOT, "include", "sg.h")).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(sg_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(sg_[a-z0-9_]+)\s*\(", text)))
 
 
 def test_header_declares_the_boundary():

@@ -273,3 +273,80 @@ def test_tensor_core_attention_matches_cuda_core_attention(dev, weights, B, M, N
         out.append(S.double().cpu().numpy())
         m.close()
     assert np.abs(out[0] - out[1]).max() < 2e-2 * max(1.0, np.abs(out[1]).max() / 10)
+
+
+@pytest.mark.gpu
+def test_fma_pipe_exp2_against_float64_and_cuda_exp2(dev):
+    from learned_sparse_feature_b200 import binding
+    xs = np.concatenate([np.linspace(-125.0, 126.0, 200001), np.linspace(-1.0, 1.0, 4001),
+                         np.array([0.0, 0.5, -0.5, 1e-7, -1e-7, 63.5, 64.49, -124.999])]).astype(np.float32)
+    x = torch.from_numpy(xs).to(dev)
+    y = torch.empty_like(x)
+    binding.selftest_exp2_poly(x, y)
+    torch.cuda.synchronize()
+    got = y.double().cpu().numpy()
+    ref = np.exp2(xs.astype(np.float64))
+    rel = np.abs(got / ref - 1.0)
+    assert rel.max() < 1e-4, (rel.max(), xs[rel.argmax()])
+    # and against CUDA's own exp2 (fp32) on the same inputs
+    cu = torch.exp2(x).double().cpu().numpy()
+    assert np.abs(got / cu - 1.0).max() < 1.1e-4
+    # clamping: far outside [-125, 126] the result saturates at the clamp values
+    xo = torch.tensor([-1e4, -300.0, 300.0, 1e4, float("-inf")], device=dev)
+    yo = torch.empty_like(xo)
+    binding.selftest_exp2_poly(xo, yo)
+    torch.cuda.synchronize()
+    vo = yo.double().cpu().numpy()
+    assert np.all(np.abs(vo[[0, 1, 4]] / 2.0 ** -125 - 1) < 1e-4)
+    assert np.all(np.abs(vo[[2, 3]] / 2.0 ** 126 - 1) < 1e-4)
+    # odd length: the last element is computed, nothing past it is written
+    x3 = torch.tensor([1.0, 2.0, 3.0], device=dev)
+    y3 = torch.full((4,), -7.0, device=dev)
+    binding.selftest_exp2_poly(x3, y3[:3])
+    torch.cuda.synchronize()
+    v3 = y3.cpu().numpy()
+    assert np.allclose(v3[:3], [2.0, 4.0, 8.0], rtol=1e-4) and v3[3] == -7.0
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("emu", ["0", "2", "4"])
+def test_attention_exp_share_variants_agree(dev, weights, emu, monkeypatch):
+    # the split of exponentials between MUFU and FMA pipe changes rounding only
+    B, M, N = 2, 200, 333
+    batch = _random_batch(B, M, N, seed=4242)
+    t = {k: torch.from_numpy(v).to(dev) for k, v in batch.items()}
+    out = []
+    for share in ("3", emu):
+        monkeypatch.setenv("SG_ATTN_EXP_EMU", share)
+        m = _matcher(weights, B, M, N, "bf16", n_stages=2)
+        S = torch.empty((B, M, N), device=dev)
+        m.scores(t["kpts0"], t["conf0"], t["desc0"], t["kpts1"], t["conf1"], t["desc1"], S)
+        assert m.status() == 0
+        out.append(S.double().cpu().numpy())
+        m.close()
+    assert np.abs(out[0] - out[1]).max() < 2e-2 * max(1.0, np.abs(out[1]).max() / 10)
+    for b in range(B):
+        ref = _oracle(batch, weights, b, n_stages=2)["scores"]
+        assert np.abs(out[1][b] - ref).max() < 5e-2
+
+
+@pytest.mark.gpu
+def test_attention_max_renewal_path(dev, weights, monkeypatch):
+    # with the bound on a tile's sum lowered to 1, nearly every key tile renews
+    # its rows' reference max and rescales the TMEM output rows; the result must
+    # not change beyond rounding
+    B, M, N = 1, 300, 700
+    batch = _random_batch(B, M, N, seed=777)
+    t = {k: torch.from_numpy(v).to(dev) for k, v in batch.items()}
+    out = []
+    for lim in ("64", "0"):
+        monkeypatch.setenv("SG_ATTN_BLIND_LIMIT_LOG2", lim)
+        m = _matcher(weights, B, M, N, "bf16", n_stages=2)
+        S = torch.empty((B, M, N), device=dev)
+        m.scores(t["kpts0"], t["conf0"], t["desc0"], t["kpts1"], t["conf1"], t["desc1"], S)
+        assert m.status() == 0
+        out.append(S.double().cpu().numpy())
+        m.close()
+    assert np.abs(out[0] - out[1]).max() < 2e-2 * max(1.0, np.abs(out[1]).max() / 10)
+    ref = _oracle(batch, weights, 0, n_stages=2)["scores"]
+    assert np.abs(out[1][0] - ref).max() < 5e-2
