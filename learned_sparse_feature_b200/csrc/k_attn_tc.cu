@@ -395,7 +395,7 @@ cudaError_t launch_attention_tc(const AttnArgs& a, cudaStream_t s, unsigned* sta
   CUtensorMap tm;
   if (!make_bf16_map(&tm, a.qkv, R, kQKV, kQKV, 128)) return cudaErrorInvalidValue;
   // share of the exponentials taken on the FMA pipe: exp_emu of every 8 pairs
-  const int emu = (a.exp_emu == 0 || a.exp_emu == 2 || a.exp_emu == 4) ? a.exp_emu : 3;
+  const int emu = (a.exp_emu == 2 || a.exp_emu == 3 || a.exp_emu == 4) ? a.exp_emu : 0;
   using Kern = void (*)(const CUtensorMap, AttnTcArgs);
   Kern kern = emu == 0 ? attn_tc_kernel<0> : emu == 2 ? attn_tc_kernel<2> : emu == 4 ? attn_tc_kernel<4>
                                                                                  : attn_tc_kernel<3>;

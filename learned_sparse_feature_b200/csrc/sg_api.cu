@@ -495,10 +495,12 @@ sg_status_t sg_create(const sg_weights* w, const sg_config* cfg, sg_handle** out
   h->use_tc = h->bf16 && tc_available() && std::getenv("SG_FORCE_SIMT") == nullptr;
   h->use_tc_attn = h->use_tc && std::getenv("SG_SIMT_ATTENTION") == nullptr;
   {
-    // SG_ATTN_EXP_EMU=0|2|3|4 overrides the default share (3 of 8); for tests
+    // SG_ATTN_EXP_EMU=2|3|4 moves that many of every 8 exp2 pairs of the
+    // attention softmax to the FMA pipe (default 0: all on the MUFU, measured
+    // fastest at these shapes); for tests and tuning
     const char* e = std::getenv("SG_ATTN_EXP_EMU");
-    const int v = e ? std::atoi(e) : 3;
-    h->attn_exp_emu = (v == 0 || v == 2 || v == 4) ? v : 3;
+    const int v = e ? std::atoi(e) : 0;
+    h->attn_exp_emu = (v == 2 || v == 3 || v == 4) ? v : 0;
     // SG_ATTN_BLIND_LIMIT_LOG2=x (0 <= x <= 64) lowers the 2^64 bound so that
     // the max-renewal path runs on ordinary inputs; for tests
     const char* b = std::getenv("SG_ATTN_BLIND_LIMIT_LOG2");

@@ -309,14 +309,14 @@ def test_fma_pipe_exp2_against_float64_and_cuda_exp2(dev):
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("emu", ["0", "2", "4"])
+@pytest.mark.parametrize("emu", ["2", "3", "4"])
 def test_attention_exp_share_variants_agree(dev, weights, emu, monkeypatch):
     # the split of exponentials between MUFU and FMA pipe changes rounding only
     B, M, N = 2, 200, 333
     batch = _random_batch(B, M, N, seed=4242)
     t = {k: torch.from_numpy(v).to(dev) for k, v in batch.items()}
     out = []
-    for share in ("3", emu):
+    for share in ("0", emu):
         monkeypatch.setenv("SG_ATTN_EXP_EMU", share)
         m = _matcher(weights, B, M, N, "bf16", n_stages=2)
         S = torch.empty((B, M, N), device=dev)
