@@ -15,19 +15,22 @@
 // owns one pair at a time; its CTAs split the M+1 rows into contiguous bands
 // and keep as many band rows as fit in shared memory, pre-scaled by log2(e)
 // and padded with -inf to LDW = 128*NQ columns, for all T iterations (the rest
-// are re-read from L2).  Inside a CTA each warp owns whole rows: lane l holds
-// the float4 column groups q*32 + l (q < NQ) of a row, and lane 0 the dustbin
-// column, so a row's reductions are warp shuffles and the per-row bookkeeping
-// is paid once per warp, not once per thread.  The column potentials live in
-// shared memory (one copy per CTA).
+// are re-read from L2).  Inside a CTA a team of SPLIT warps owns whole rows
+// (8 teams): warp h of a team holds the float4 column groups q*32 + l,
+// h*NQ/SPLIT <= q < (h+1)*NQ/SPLIT, of a row in lane l, and lane 0 of warp 0
+// the dustbin column; a row's reductions are warp shuffles plus, with
+// SPLIT > 1, one exchange of the warps' partials through shared memory under
+// a named barrier of the team.  Splitting rows keeps the per-thread state
+// small enough for 256*SPLIT threads, whose latency hiding the MUFU-bound row
+// pass needs.  The column potentials live in shared memory (one copy per CTA).
 //
 // One iteration:
-//   row pass (warp-local): each row's LSE with the shift m_r = log mu_r - u_r
+//   row pass (team-local): each row's LSE with the shift m_r = log mu_r - u_r
 //     (the row's previous LSE; the exact max on the first iteration), one MUFU
 //     ex2 per element; the same exponentials scaled by mu_r / rowsum_r are the
 //     plan mass P_rj = exp(Z + u + v) that the column update needs, summed per
-//     column in registers and then across the CTA's warps with shared-memory
-//     atomics;
+//     column in registers and then across the CTA's teams by a tree through
+//     shared memory;
 //   column pass: with cpp == 1 the CTA's column sums are final; otherwise
 //     every CTA adds its whole column vector to a global accumulator with ONE
 //     bulk asynchronous reduction (cp.reduce.async.bulk ... add.f32), the group
@@ -37,7 +40,7 @@
 // precision could have been lost to underflow) that LSE is recomputed exactly
 // with its true max.  Every decision that steers control flow is taken on
 // values that are identical in all the threads that have to agree on it (rows:
-// the warp; columns: the whole group).
+// the team; columns: the whole group).
 //
 // Waits: the group barrier spins with a time limit and, on expiry, latches a
 // timeout in the status word, raises an abort flag that ends every other
@@ -53,8 +56,7 @@
 namespace sg {
 namespace {
 
-constexpr int NT = 256;
-constexpr int NWARP = NT / 32;
+constexpr int NTEAM = 8;                 // row teams per CTA
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRowTiny = 9.094947017729282e-13f;   // 2^-40
@@ -169,15 +171,26 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 }
 
 // ------------------------------------------------------------------ kernel
-template <int NQ>
-__global__ void __launch_bounds__(NT, 1) sinkhorn_kernel(SinkhornArgs a) {
-  constexpr int CPL = 4 * NQ;                     // columns per lane
+// Named barrier of the SPLIT warps of team t (ids 1..8; 0 is __syncthreads).
+template <int SPLIT>
+__device__ __forceinline__ void team_sync(int t) {
+  if (SPLIT > 1) asm volatile("bar.sync %0, %1;" ::"r"(1 + t), "n"(32 * SPLIT) : "memory");
+}
+
+template <int NQ, int SPLIT>
+__global__ void __launch_bounds__(256 * SPLIT, 1) sinkhorn_kernel(SinkhornArgs a) {
+  constexpr int NT = 256 * SPLIT;
+  constexpr int NWARP = NT / 32;
+  constexpr int NQW = NQ / SPLIT;                 // float4 groups per lane (one warp's share of a row)
+  constexpr int CPW = 4 * NQW;                    // columns per lane
+  static_assert(NQ % SPLIT == 0 && NWARP == NTEAM * SPLIT, "row split");
   constexpr int LDW = 128 * NQ;                   // padded row length
   constexpr int CV = LDW + 4;                     // column vector (+ dustbin at LDW)
   extern __shared__ __align__(16) unsigned char smraw[];
 
   const int tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5;
+  const int team = warp % NTEAM, part = warp / NTEAM;   // row team, share of the row
   const int cpp = a.cpp;
   const int group = blockIdx.x / cpp;
   const int rank = blockIdx.x % cpp;
@@ -190,13 +203,15 @@ __global__ void __launch_bounds__(NT, 1) sinkhorn_kernel(SinkhornArgs a) {
   const int cached = min(r1 - r0, a.cached_rows);
 
   // shared memory: [cache rows x LDW | v (CV) | column totals (CV) |
-  //                 warp partials (NWARP/2 x CV) | u (band)]
+  //                 team partials (NTEAM/2 x CV) | u (band)]
   float* cache = reinterpret_cast<float*>(smraw);
   float* vbuf = cache + (size_t)a.cached_rows * LDW;
   float* ctot = vbuf + CV;
   unsigned* ckey = reinterpret_cast<unsigned*>(ctot);
-  float* xbuf = ctot + CV;                        // NWARP/2 partial column vectors
-  float* u2s = xbuf + (size_t)(NWARP / 2) * CV;
+  float* xbuf = ctot + CV;                        // NTEAM/2 partial column vectors
+  float* u2s = xbuf + (size_t)(NTEAM / 2) * CV;
+  // per team and row parity: the parts' partial maxima and sums of a row
+  __shared__ float xr_max[2][NTEAM][SPLIT], xr_sum[2][NTEAM][SPLIT];
   // extraction only: per-column best (value, row) keys over the row cache
   unsigned long long* cbest = reinterpret_cast<unsigned long long*>(smraw);
 
@@ -226,19 +241,20 @@ __global__ void __launch_bounds__(NT, 1) sinkhorn_kernel(SinkhornArgs a) {
     float* fbs = fbm + Cp;                         // exact column fallback: sums
     unsigned* fbk = reinterpret_cast<unsigned*>(fbm);
 
-    // z2 (log2 domain) of row r, from the source matrix, for this lane's groups
-    auto load_src = [&](int r, float (&z)[CPL]) {
+    // z2 (log2 domain) of row r, from the source matrix, for this lane's float4
+    // groups g0 .. g0 + NQW - 1
+    auto load_src = [&](int r, int g0, float (&z)[CPW]) {
       if (r == M) {
 #pragma unroll
-        for (int q = 0; q < NQ; ++q)
+        for (int qq = 0; qq < NQW; ++qq)
 #pragma unroll
-          for (int i = 0; i < 4; ++i) z[4 * q + i] = (q * 128 + lane * 4 + i) < N ? alpha2 : -INFINITY;
+          for (int i = 0; i < 4; ++i) z[4 * qq + i] = ((g0 + qq) * 128 + lane * 4 + i) < N ? alpha2 : -INFINITY;
         return;
       }
       const float* src = S + (long long)r * a.lds;
 #pragma unroll
-      for (int q = 0; q < NQ; ++q) {
-        const int o = q * 128 + lane * 4;
+      for (int qq = 0; qq < NQW; ++qq) {
+        const int o = (g0 + qq) * 128 + lane * 4;
         float4 t = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
         if (a.lds_vec && o + 3 < N) {
           t = __ldg(reinterpret_cast<const float4*>(src + o));
@@ -249,20 +265,20 @@ __global__ void __launch_bounds__(NT, 1) sinkhorn_kernel(SinkhornArgs a) {
           if (o + 2 < N) t.z = __ldg(src + o + 2) * kLog2e;
           if (o + 3 < N) t.w = __ldg(src + o + 3) * kLog2e;
         }
-        z[4 * q] = t.x; z[4 * q + 1] = t.y; z[4 * q + 2] = t.z; z[4 * q + 3] = t.w;
+        z[4 * qq] = t.x; z[4 * qq + 1] = t.y; z[4 * qq + 2] = t.z; z[4 * qq + 3] = t.w;
       }
     };
     // z2 of row r: from the shared-memory cache when the row is cached
-    auto load_row = [&](int r, float (&z)[CPL]) {
+    auto load_row = [&](int r, int g0, float (&z)[CPW]) {
       if (r - r0 < cached) {
         const float4* row = reinterpret_cast<const float4*>(cache + (size_t)(r - r0) * LDW);
 #pragma unroll
-        for (int q = 0; q < NQ; ++q) {
-          const float4 t = row[q * 32 + lane];
-          z[4 * q] = t.x; z[4 * q + 1] = t.y; z[4 * q + 2] = t.z; z[4 * q + 3] = t.w;
+        for (int qq = 0; qq < NQW; ++qq) {
+          const float4 t = row[(g0 + qq) * 32 + lane];
+          z[4 * qq] = t.x; z[4 * qq + 1] = t.y; z[4 * qq + 2] = t.z; z[4 * qq + 3] = t.w;
         }
       } else {
-        load_src(r, z);
+        load_src(r, g0, z);
       }
     };
     // ---- stage the band in shared memory (pre-scaled, padded with -inf)
@@ -278,85 +294,108 @@ __global__ void __launch_bounds__(NT, 1) sinkhorn_kernel(SinkhornArgs a) {
     __syncthreads();
 
     for (int it = 0; it < a.iters; ++it) {
-      // ------------------------------------------------ row pass (warp per row)
-      float colacc[CPL];
+      // ------------------------------------------------ row pass (team per row)
+      float colacc[CPW];
 #pragma unroll
-      for (int c = 0; c < CPL; ++c) colacc[c] = 0.f;
+      for (int c = 0; c < CPW; ++c) colacc[c] = 0.f;
       float colbin = 0.f;
       const float4* v4 = reinterpret_cast<const float4*>(vbuf);   // read in the loop: saves registers
       const float vb = vbuf[LDW];
-      for (int r = r0 + warp; r < r1; r += NWARP) {
+      const int g0 = part * NQW;                  // this warp's first float4 group
+      const bool bin_lane = part == 0 && lane == 0;
+      int k = 0;                                  // rows taken by the team (slot parity)
+      for (int r = r0 + team; r < r1; r += NTEAM, ++k) {
         const float lmu2 = r < M ? lmu_r2 : lmu_b2;
-        float e[CPL];
-        load_row(r, e);
+        float e[CPW];
+        load_row(r, g0, e);
         bool exact = (it == 0);
         float m = exact ? 0.f : lmu2 - u2[r];
         float s, eb;
         while (true) {
           if (exact) {
-            float mx = lane == 0 ? alpha2 + vb : -INFINITY;
+            float mx = bin_lane ? alpha2 + vb : -INFINITY;
 #pragma unroll
-            for (int q = 0; q < NQ; ++q) {
-              const float4 vq = v4[q * 32 + lane];
-              mx = fmaxf(mx, fmaxf(fmaxf(e[4 * q] + vq.x, e[4 * q + 1] + vq.y),
-                                   fmaxf(e[4 * q + 2] + vq.z, e[4 * q + 3] + vq.w)));
+            for (int qq = 0; qq < NQW; ++qq) {
+              const float4 vq = v4[(g0 + qq) * 32 + lane];
+              mx = fmaxf(mx, fmaxf(fmaxf(e[4 * qq] + vq.x, e[4 * qq + 1] + vq.y),
+                                   fmaxf(e[4 * qq + 2] + vq.z, e[4 * qq + 3] + vq.w)));
             }
             m = warp_max(mx);
-          }
-          float part = 0.f;
+            if (SPLIT > 1) {
+              if (lane == 0) xr_max[k & 1][team][part] = m;
+              team_sync<SPLIT>(team);
+              m = xr_max[k & 1][team][0];
 #pragma unroll
-          for (int q = 0; q < NQ; ++q) {
-            const float4 vq = v4[q * 32 + lane];
-            const float x0 = ex2((e[4 * q] + vq.x) - m);
-            const float x1 = ex2((e[4 * q + 1] + vq.y) - m);
-            const float x2 = ex2((e[4 * q + 2] + vq.z) - m);
-            const float x3 = ex2((e[4 * q + 3] + vq.w) - m);
-            e[4 * q] = x0; e[4 * q + 1] = x1; e[4 * q + 2] = x2; e[4 * q + 3] = x3;
-            part += (x0 + x1) + (x2 + x3);
+              for (int h = 1; h < SPLIT; ++h) m = fmaxf(m, xr_max[k & 1][team][h]);
+            }
           }
-          eb = lane == 0 ? ex2((alpha2 + vb) - m) : 0.f;
-          s = warp_sum(part + eb);
-          if (exact || (s >= kRowTiny && s < INFINITY)) break;   // warp-uniform
+          float part_s = 0.f;
+#pragma unroll
+          for (int qq = 0; qq < NQW; ++qq) {
+            const float4 vq = v4[(g0 + qq) * 32 + lane];
+            const float x0 = ex2((e[4 * qq] + vq.x) - m);
+            const float x1 = ex2((e[4 * qq + 1] + vq.y) - m);
+            const float x2 = ex2((e[4 * qq + 2] + vq.z) - m);
+            const float x3 = ex2((e[4 * qq + 3] + vq.w) - m);
+            e[4 * qq] = x0; e[4 * qq + 1] = x1; e[4 * qq + 2] = x2; e[4 * qq + 3] = x3;
+            part_s += (x0 + x1) + (x2 + x3);
+          }
+          eb = bin_lane ? ex2((alpha2 + vb) - m) : 0.f;
+          s = warp_sum(part_s + eb);
+          if (SPLIT > 1) {
+            // every part adds the same partials in the same order: s is
+            // identical in the whole team
+            if (lane == 0) xr_sum[k & 1][team][part] = s;
+            team_sync<SPLIT>(team);
+            s = xr_sum[k & 1][team][0];
+#pragma unroll
+            for (int h = 1; h < SPLIT; ++h) s += xr_sum[k & 1][team][h];
+          }
+          if (exact || (s >= kRowTiny && s < INFINITY)) break;   // team-uniform
           exact = true;                           // reload the raw row and redo it exactly
-          load_row(r, e);
+          load_row(r, g0, e);
+          ++k;                                    // fresh exchange slots for the redo
         }
         const float ls = lg2(s);
         const float ratio = ex2(lmu2 - ls);       // mu_r / rowsum_r
-        if (lane == 0) u2[r] = lmu2 - m - ls;
+        if (bin_lane) u2[r] = lmu2 - m - ls;
 #pragma unroll
-        for (int c = 0; c < CPL; ++c) colacc[c] = fmaf(e[c], ratio, colacc[c]);
+        for (int c = 0; c < CPW; ++c) colacc[c] = fmaf(e[c], ratio, colacc[c]);
         colbin = fmaf(eb, ratio, colbin);
       }
-      // CTA column sums: a 3-round tree over the warps through shared memory
-      // (8 -> 4 -> 2 -> 1 partial vectors; shared fp32 atomics from 8 warps on
-      // the same addresses are an order of magnitude slower)
+      // CTA column sums: a 3-round tree over the teams through shared memory
+      // (8 -> 4 -> 2 -> 1 partial vectors; the parts of a team own disjoint
+      // columns of the same vectors; shared fp32 atomics from 8 warps on the
+      // same addresses are an order of magnitude slower)
 #pragma unroll
-      for (int half = NWARP / 2; half >= 1; half >>= 1) {
-        if (warp >= half && warp < 2 * half) {
-          float4* dst = reinterpret_cast<float4*>(xbuf + (size_t)(warp - half) * CV);
+      for (int half = NTEAM / 2; half >= 1; half >>= 1) {
+        if (team >= half && team < 2 * half) {
+          float4* dst = reinterpret_cast<float4*>(xbuf + (size_t)(team - half) * CV);
 #pragma unroll
-          for (int q = 0; q < NQ; ++q)
-            dst[q * 32 + lane] = make_float4(colacc[4 * q], colacc[4 * q + 1], colacc[4 * q + 2], colacc[4 * q + 3]);
-          if (lane == 0) xbuf[(size_t)(warp - half) * CV + LDW] = colbin;
+          for (int qq = 0; qq < NQW; ++qq)
+            dst[(g0 + qq) * 32 + lane] =
+                make_float4(colacc[4 * qq], colacc[4 * qq + 1], colacc[4 * qq + 2], colacc[4 * qq + 3]);
+          if (bin_lane) xbuf[(size_t)(team - half) * CV + LDW] = colbin;
         }
         __syncthreads();
-        if (warp < half) {
-          const float4* src = reinterpret_cast<const float4*>(xbuf + (size_t)warp * CV);
+        if (team < half) {
+          const float4* src = reinterpret_cast<const float4*>(xbuf + (size_t)team * CV);
 #pragma unroll
-          for (int q = 0; q < NQ; ++q) {
-            const float4 t = src[q * 32 + lane];
-            colacc[4 * q] += t.x; colacc[4 * q + 1] += t.y; colacc[4 * q + 2] += t.z; colacc[4 * q + 3] += t.w;
+          for (int qq = 0; qq < NQW; ++qq) {
+            const float4 t = src[(g0 + qq) * 32 + lane];
+            colacc[4 * qq] += t.x; colacc[4 * qq + 1] += t.y; colacc[4 * qq + 2] += t.z; colacc[4 * qq + 3] += t.w;
           }
-          if (lane == 0) colbin += xbuf[(size_t)warp * CV + LDW];
+          if (bin_lane) colbin += xbuf[(size_t)team * CV + LDW];
         }
         __syncthreads();
       }
-      if (warp == 0) {
+      if (team == 0) {
         float4* dst = reinterpret_cast<float4*>(ctot);
 #pragma unroll
-        for (int q = 0; q < NQ; ++q)
-          dst[q * 32 + lane] = make_float4(colacc[4 * q], colacc[4 * q + 1], colacc[4 * q + 2], colacc[4 * q + 3]);
-        if (lane == 0) ctot[LDW] = colbin;
+        for (int qq = 0; qq < NQW; ++qq)
+          dst[(g0 + qq) * 32 + lane] =
+              make_float4(colacc[4 * qq], colacc[4 * qq + 1], colacc[4 * qq + 2], colacc[4 * qq + 3]);
+        if (bin_lane) ctot[LDW] = colbin;
       }
       __syncthreads();
       // ------------------------------------------------ column pass (group)
@@ -393,16 +432,18 @@ __global__ void __launch_bounds__(NT, 1) sinkhorn_kernel(SinkhornArgs a) {
         for (int j = tid; j < CV; j += NT) ckey[j] = 0u;
         __syncthreads();
         for (int r = r0 + warp; r < r1; r += NWARP) {
-          float z[CPL];
-          load_row(r, z);
           const float ur = u2[r];
+          for (int h = 0; h < SPLIT; ++h) {
+            float z[CPW];
+            load_row(r, h * NQW, z);
 #pragma unroll
-          for (int q = 0; q < NQ; ++q)
+            for (int qq = 0; qq < NQW; ++qq)
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const int j = q * 128 + lane * 4 + i;
-              if (j < N) atomicMax(ckey + j, f2key(z[4 * q + i] + ur));
-            }
+              for (int i = 0; i < 4; ++i) {
+                const int j = (h * NQW + qq) * 128 + lane * 4 + i;
+                if (j < N) atomicMax(ckey + j, f2key(z[4 * qq + i] + ur));
+              }
+          }
           if (lane == 0) atomicMax(ckey + LDW, f2key(alpha2 + ur));
         }
         __syncthreads();
@@ -413,18 +454,20 @@ __global__ void __launch_bounds__(NT, 1) sinkhorn_kernel(SinkhornArgs a) {
         for (int j = tid; j < CV; j += NT) { vbuf[j] = key2f(__ldcg(fbk + j)); ctot[j] = 0.f; }
         __syncthreads();
         for (int r = r0 + warp; r < r1; r += NWARP) {
-          float z[CPL];
-          load_row(r, z);
           const float ur = u2[r];
           const float4* mx4 = reinterpret_cast<const float4*>(vbuf);
+          for (int h = 0; h < SPLIT; ++h) {
+            float z[CPW];
+            load_row(r, h * NQW, z);
 #pragma unroll
-          for (int q = 0; q < NQ; ++q) {
-            const float4 mq = mx4[q * 32 + lane];
-            const float mm[4] = {mq.x, mq.y, mq.z, mq.w};
+            for (int qq = 0; qq < NQW; ++qq) {
+              const float4 mq = mx4[(h * NQW + qq) * 32 + lane];
+              const float mm[4] = {mq.x, mq.y, mq.z, mq.w};
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const int j = q * 128 + lane * 4 + i;
-              if (j < N) atomicAdd(ctot + j, ex2((z[4 * q + i] + ur) - mm[i]));
+              for (int i = 0; i < 4; ++i) {
+                const int j = (h * NQW + qq) * 128 + lane * 4 + i;
+                if (j < N) atomicAdd(ctot + j, ex2((z[4 * qq + i] + ur) - mm[i]));
+              }
             }
           }
           if (lane == 0) atomicAdd(ctot + LDW, ex2((alpha2 + ur) - vbuf[LDW]));
@@ -462,20 +505,22 @@ __global__ void __launch_bounds__(NT, 1) sinkhorn_kernel(SinkhornArgs a) {
     unsigned long long* cb = a.colbest + (long long)pair * N;
     float* lp = a.logP ? a.logP + (long long)pair * R * C : nullptr;
     for (int r = r0 + warp; r < r1; r += NWARP) {
-      float z[CPL];
-      load_src(r, z);
       const float ur = u2[r];
       if (!isfinite(ur)) nonfinite = true;
       unsigned long long best = 0ull;
+      for (int h = 0; h < SPLIT; ++h) {
+      float z[CPW];
+      load_src(r, h * NQW, z);
 #pragma unroll
-      for (int q = 0; q < NQ; ++q) {
+      for (int qq = 0; qq < NQW; ++qq) {
+        const int q = h * NQW + qq;
         const float4 vq = v4[q * 32 + lane];
         const float vv[4] = {vq.x, vq.y, vq.z, vq.w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int j = q * 128 + lane * 4 + i;
           if (j >= N) continue;
-          const float val = ((z[4 * q + i] + ur) + vv[i]) * kLn2 - norm;
+          const float val = ((z[4 * qq + i] + ur) + vv[i]) * kLn2 - norm;
           if (lp) lp[(long long)r * C + j] = val;
           if (r < M) {
             const unsigned long long kr = ((unsigned long long)f2key(val) << 32) | (0xffffffffu - (unsigned)j);
@@ -485,6 +530,7 @@ __global__ void __launch_bounds__(NT, 1) sinkhorn_kernel(SinkhornArgs a) {
             else atomicMax(cb + j, kc);
           }
         }
+      }
       }
       if (lane == 0 && lp) lp[(long long)r * C + N] = ((alpha2 + ur) + vb) * kLn2 - norm;
       if (r < M) {
@@ -539,25 +585,31 @@ __global__ void barrier_selftest_kernel(unsigned* counter, unsigned* abort_flag,
 }
 
 // ------------------------------------------------------------------ host side
+// Warps per row: one for short rows; for long rows two (three for the longest),
+// so that the per-thread row state stays small enough for 512 (768) threads.
+template <int NQ> struct SplitOf { static constexpr int value = NQ >= 24 ? 3 : NQ >= 8 ? 2 : 1; };
+
 template <int NQ>
 cudaError_t prepare() {
   static bool done = false;
   if (done) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(sinkhorn_kernel<NQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)kMaxSmem);
+  cudaError_t e = cudaFuncSetAttribute(sinkhorn_kernel<NQ, SplitOf<NQ>::value>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kMaxSmem);
   if (e == cudaSuccess) done = true;
   return e;
 }
 
 template <int NQ>
 cudaError_t launch_t(SinkhornArgs a, int num_sms, cudaStream_t s, int* launches) {
-  auto kern = sinkhorn_kernel<NQ>;
+  constexpr int SPLIT = SplitOf<NQ>::value;
+  constexpr int NT = 256 * SPLIT;
+  auto kern = sinkhorn_kernel<NQ, SPLIT>;
   constexpr int LDW = 128 * NQ;
   constexpr int CV = LDW + 4;
   cudaError_t e = prepare<NQ>();
   if (e != cudaSuccess) return e;
   const int R = a.M + 1;
-  const size_t fixed = (2 + NWARP / 2) * (size_t)CV * 4;
+  const size_t fixed = (2 + NTEAM / 2) * (size_t)CV * 4;
   const double clk = 1.9e9;
   const double pair_bytes = (double)R * a.N * 4;
   // CTAs per pair, from a cost model of one iteration: MUFU ex2 and issue
