@@ -12,7 +12,10 @@
 //                      one of two 128 x BN fp32 accumulators in TMEM;
 //                      tcgen05.commit frees the stage / publishes the tile;
 //   warps 2-5          epilogue: tcgen05.ld of the thread's accumulator row (TMEM
-//                      lane = tile row), bias / ReLU / residual / scale, store,
+//                      lane = tile row), bias / ReLU / residual / scale, written as
+//                      a 32 x 32 chunk into swizzled shared memory and stored by
+//                      one TMA tensor store per chunk (double-buffered; the
+//                      residual comes in by TMA tensor loads two chunks ahead),
 //                      while the MMA warp already fills the other accumulator.
 // Launched with programmatic dependent launch: the prologue (barriers, TMEM,
 // descriptor prefetch) overlaps the previous kernel; griddepcontrol.wait gates
@@ -49,12 +52,36 @@ struct TcArgs {
   unsigned* status;
 };
 
-template <int BN, int STAGES>
+// Epilogue staging of one epilogue warp: two buffer sets, each a 32-row chunk of
+// the output (fp32 rows of 128 B or bf16 rows of 64 B) and, for the residual
+// epilogue, its bf16 copy and the fp32 residual input.  Offsets are multiples
+// of 1024 B (the swizzle atoms of the TMA boxes).
+template <int EPI>
+struct EpiStage {
+  static constexpr bool F32 = EPI == EPI_SCALE || EPI == EPI_RESIDUAL;
+  static constexpr int OUT = F32 ? 4096 : 2048;
+  static constexpr int OUT2 = EPI == EPI_RESIDUAL ? 2048 : 0;
+  static constexpr int RES = EPI == EPI_RESIDUAL ? 4096 : 0;
+  static constexpr int OUT2_OFF = OUT;
+  static constexpr int RES_OFF = OUT + OUT2;
+  static constexpr int BUF = OUT + OUT2 + RES;
+  static constexpr int WARP = 2 * BUF;
+  static constexpr int BYTES = 4 * WARP;
+};
+
+constexpr int kMaxDynSmem = 224 * 1024;
+
+template <int BN, int EPI>
 struct Smem {
   static constexpr int A_BYTES = BM * BK * 2;
   static constexpr int B_BYTES = BN * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int BYTES = STAGES * STAGE_BYTES + 1024;   // + alignment slack
+  // as many ring stages as fit next to the epilogue staging (at most 8)
+  static constexpr int FIT = (kMaxDynSmem - EpiStage<EPI>::BYTES - 1024) / STAGE_BYTES;
+  static constexpr int STAGES = FIT > 8 ? 8 : FIT;
+  static constexpr int EPI_OFF = STAGES * STAGE_BYTES;
+  static constexpr int BYTES = EPI_OFF + EpiStage<EPI>::BYTES + 1024;   // + alignment slack
+  static_assert(STAGES >= 2, "shared memory");
 };
 
 template <int BN> __host__ __device__ constexpr uint32_t tmem_cols() {
@@ -84,17 +111,21 @@ __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.lau
 // consecutive CTAs share the A tile in L2.  The accumulator is double-buffered
 // in TMEM: the epilogue warps drain tile i while the MMA warp accumulates tile
 // i + 1.
-template <int BN, int STAGES, int EPI>
+template <int BN, int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
-               const __grid_constant__ CUtensorMap tmB, TcArgs g) {
-  using SM = Smem<BN, STAGES>;
+               const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmO,
+               const __grid_constant__ CUtensorMap tmO2, TcArgs g) {
+  using SM = Smem<BN, EPI>;
+  using ES = EpiStage<EPI>;
+  constexpr int STAGES = SM::STAGES;
   constexpr uint32_t BNA = tmem_cols<BN>();      // TMEM columns of one accumulator buffer
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[STAGES];
   __shared__ __align__(8) uint64_t empty_bar[STAGES];
   __shared__ __align__(8) uint64_t tfull_bar[2];
   __shared__ __align__(8) uint64_t tempty_bar[2];
+  __shared__ __align__(8) uint64_t res_bar[4][2];   // residual chunk loads, per epilogue warp and buffer
   __shared__ __align__(16) float s_bias[2][BN];   // bias of the tile, by accumulator buffer
   __shared__ uint32_t tmem_slot;
   __shared__ int s_abort;
@@ -119,6 +150,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
       tc::mbar_init(&tfull_bar[b], 1);
       tc::mbar_init(&tempty_bar[b], 4);          // one arrival per epilogue warp
     }
+    for (int w = 0; w < 4; ++w) {
+      tc::mbar_init(&res_bar[w][0], 1);
+      tc::mbar_init(&res_bar[w][1], 1);
+    }
     tc::fence_barrier_init();
     s_abort = 0;
   }
@@ -127,6 +162,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
     tc::prefetch_tmap(&tmA0);
     tc::prefetch_tmap(&tmA1);
     tc::prefetch_tmap(&tmB);
+    tc::prefetch_tmap(&tmO);
+    if (EPI == EPI_RESIDUAL) tc::prefetch_tmap(&tmO2);
   }
   tc::tc_fence_before();
   __syncthreads();
@@ -202,27 +239,31 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
   } else {
     // ---------------- epilogue warps 2..5: TMEM lane quarter = warp % 4
     // While the MMA warp accumulates a tile, these warps stage its bias in
-    // shared memory and start the loads of its first residual chunk, so that no
-    // global-memory latency sits between the accumulator and the stores.
+    // shared memory and (residual) start the TMA loads of the first two
+    // residual chunks.  Warp q owns tile rows 32q .. 32q+31, thread = row.
     const int q = warp & 3;
     const int et = threadIdx.x - 64;             // 0..127
+    uint8_t* wbuf = sbase + SM::EPI_OFF + q * ES::WARP;
+    constexpr int NCH = BN / 32;                 // 32-column chunks per tile
+    int chunk = 0;                               // chunks done by this warp (buffer = chunk & 1)
+    uint32_t res_par = 0;                        // residual barrier parities, bit per buffer
+    uint32_t res_pend = 0;                       // residual loads issued and not yet waited for
     int i = 0;
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++i) {
       const int b = i & 1;
       const int tn = t % ntn, tm = (t / ntn) % ntm, bz = t / (ntn * ntm);
       const int n0 = tn * BN;
-      const int row = tm * BM + q * 32 + lane;
-      const bool row_ok = row < g.rows;
-      const long long rbase = (long long)bz * g.strideO + (long long)row * g.ldo + n0;
+      const int row0 = tm * BM + q * 32;         // first row of this warp's chunks
       if (EPI == EPI_BIAS || EPI == EPI_BIAS_RELU) {
         for (int c = et; c < BN; c += 128) s_bias[b][c] = (n0 + c < g.cols) ? __ldg(g.bias + n0 + c) : 0.f;
       }
-      float4 rnext[8];
-      const bool vec_res = EPI == EPI_RESIDUAL && n0 + BN <= g.cols;   // full-width tile: float4 path
-      if (EPI == EPI_RESIDUAL && vec_res && row_ok) {
-        const float4* x4 = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(g.out) + rbase);
-#pragma unroll
-        for (int k = 0; k < 8; ++k) rnext[k] = __ldcg(x4 + k);
+      if (EPI == EPI_RESIDUAL && lane == 0) {
+        for (int c = 0; c < 2 && c < NCH; ++c) {
+          const int bb = (chunk + c) & 1;
+          tc::mbar_arrive_expect_tx(&res_bar[q][bb], 4096);
+          tc::tma_load_3d(&tmO, &res_bar[q][bb], wbuf + bb * ES::BUF + ES::RES_OFF, n0 + 32 * c, row0, bz);
+          res_pend |= 1u << bb;
+        }
       }
       const bool got = tc::mbar_wait(&tfull_bar[b], (i >> 1) & 1, g.status, kErrGemmWait);
       // one barrier of the 128 epilogue threads per tile: publishes the staged
@@ -230,99 +271,94 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
       if (!epi_all(got && !s_abort)) break;
       tc::tc_fence_after();
       const uint32_t trow = tmem + b * BNA + ((uint32_t)(q * 32) << 16);
+      bool ok = true;
 #pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += 32) {
+      for (int ci = 0; ci < NCH; ++ci, ++chunk) {
+        const int bb = chunk & 1;
+        uint8_t* sbuf = wbuf + bb * ES::BUF;
         float v[32];
-        tc::tmem_ld32(trow + c0, v);             // warp-collective: every lane takes part
-        float4 rcur[8];
-        if (EPI == EPI_RESIDUAL && vec_res) {
-#pragma unroll
-          for (int k = 0; k < 8; ++k) rcur[k] = rnext[k];
-          if (c0 + 32 < BN && row_ok) {
-            const float4* x4 = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(g.out) + rbase + c0 + 32);
-#pragma unroll
-            for (int k = 0; k < 8; ++k) rnext[k] = __ldcg(x4 + k);
-          }
-        }
-        if (!row_ok || n0 + c0 >= g.cols) continue;
-        const long long obase = rbase + c0;
-        const int ncol = min(32, g.cols - (n0 + c0));
+        tc::tmem_ld32(trow + ci * 32, v);       // warp-collective: every lane takes part
+        // the store issued from this buffer two chunks ago must have read it
+        if (lane == 0) tc::bulk_wait_read<1>();
+        __syncwarp();
         if (EPI == EPI_BIAS || EPI == EPI_BIAS_RELU) {
-          __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(g.out) + obase;
-          const float* sbv = s_bias[b] + c0;
-          if (ncol == 32) {
-            uint4 pk[4];
-            uint32_t* p = reinterpret_cast<uint32_t*>(pk);
-            const float4* b4 = reinterpret_cast<const float4*>(sbv);
+          // bf16 row of 64 B, 64-byte swizzle: 16-byte chunk k at k ^ ((row >> 1) & 3)
+          const float4* b4 = reinterpret_cast<const float4*>(s_bias[b] + ci * 32);
+          uint8_t* rowp = sbuf + lane * 64;
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
-              const float4 bb = b4[k];
-              float x0 = v[4 * k] + bb.x, x1 = v[4 * k + 1] + bb.y, x2 = v[4 * k + 2] + bb.z, x3 = v[4 * k + 3] + bb.w;
+          for (int k = 0; k < 4; ++k) {
+            uint32_t pk[4];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const float4 bb4 = b4[2 * k + h];
+              float x0 = v[8 * k + 4 * h] + bb4.x, x1 = v[8 * k + 4 * h + 1] + bb4.y;
+              float x2 = v[8 * k + 4 * h + 2] + bb4.z, x3 = v[8 * k + 4 * h + 3] + bb4.w;
               if (EPI == EPI_BIAS_RELU) {
                 x0 = fmaxf(x0, 0.f); x1 = fmaxf(x1, 0.f); x2 = fmaxf(x2, 0.f); x3 = fmaxf(x3, 0.f);
               }
-              p[2 * k] = tc::pack_bf16x2(x0, x1);
-              p[2 * k + 1] = tc::pack_bf16x2(x2, x3);
+              pk[2 * h] = tc::pack_bf16x2(x0, x1);
+              pk[2 * h + 1] = tc::pack_bf16x2(x2, x3);
             }
-            uint4* o4 = reinterpret_cast<uint4*>(o);
-#pragma unroll
-            for (int k = 0; k < 4; ++k) o4[k] = pk[k];
-          } else {
-#pragma unroll
-            for (int k = 0; k < 32; ++k) {           // static indices keep v in registers
-              if (k < ncol) {
-                float x = v[k] + sbv[k];
-                if (EPI == EPI_BIAS_RELU) x = fmaxf(x, 0.f);
-                o[k] = __float2bfloat16_rn(x);
-              }
-            }
+            *reinterpret_cast<uint4*>(rowp + ((k ^ ((lane >> 1) & 3)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
           }
-        } else if (EPI == EPI_RESIDUAL) {
-          float* x = reinterpret_cast<float*>(g.out) + obase;
-          __nv_bfloat16* xb = reinterpret_cast<__nv_bfloat16*>(g.out2) + obase;
-          if (vec_res) {
-            float4* x4 = reinterpret_cast<float4*>(x);
-            uint4 pk[4];
-            uint32_t* p = reinterpret_cast<uint32_t*>(pk);
+        } else if (EPI == EPI_SCALE) {
+          // fp32 row of 128 B, 128-byte swizzle: 16-byte chunk k at k ^ (row & 7)
+          uint8_t* rowp = sbuf + lane * 128;
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
-              float4 r = rcur[k];
-              r.x += v[4 * k]; r.y += v[4 * k + 1]; r.z += v[4 * k + 2]; r.w += v[4 * k + 3];
-              x4[k] = r;
-              p[2 * k] = tc::pack_bf16x2(r.x, r.y);
-              p[2 * k + 1] = tc::pack_bf16x2(r.z, r.w);
-            }
-            uint4* o4 = reinterpret_cast<uint4*>(xb);
-#pragma unroll
-            for (int k = 0; k < 4; ++k) o4[k] = pk[k];
-          } else {
-#pragma unroll
-            for (int k = 0; k < 32; ++k) {
-              if (k < ncol) {
-                const float r = x[k] + v[k];
-                x[k] = r;
-                xb[k] = __float2bfloat16_rn(r);
-              }
-            }
-          }
+          for (int k = 0; k < 8; ++k)
+            *reinterpret_cast<float4*>(rowp + ((k ^ (lane & 7)) << 4)) =
+                make_float4(v[4 * k] * g.scale, v[4 * k + 1] * g.scale, v[4 * k + 2] * g.scale, v[4 * k + 3] * g.scale);
         } else {
-          float* o = reinterpret_cast<float*>(g.out) + obase;
-          if (ncol == 32 && (g.ldo % 4) == 0 && (g.strideO % 4) == 0) {
-            float4* o4 = reinterpret_cast<float4*>(o);
+          // residual: x (fp32) += acc, and its bf16 copy
+          ok = tc::mbar_wait(&res_bar[q][bb], (res_par >> bb) & 1u, g.status, kErrGemmWait);
+          res_par ^= 1u << bb;
+          res_pend &= ~(1u << bb);
+          const uint8_t* rin = sbuf + ES::RES_OFF + lane * 128;
+          uint8_t* rout = sbuf + lane * 128;
+          uint8_t* rout2 = sbuf + ES::OUT2_OFF + lane * 64;
+          uint32_t pk[16];
 #pragma unroll
-            for (int k = 0; k < 8; ++k)
-              o4[k] = make_float4(v[4 * k] * g.scale, v[4 * k + 1] * g.scale, v[4 * k + 2] * g.scale,
-                                  v[4 * k + 3] * g.scale);
-          } else {
+          for (int k = 0; k < 8; ++k) {
+            const int off = (k ^ (lane & 7)) << 4;
+            float4 r = *reinterpret_cast<const float4*>(rin + off);
+            r.x += v[4 * k]; r.y += v[4 * k + 1]; r.z += v[4 * k + 2]; r.w += v[4 * k + 3];
+            *reinterpret_cast<float4*>(rout + off) = r;
+            pk[2 * k] = tc::pack_bf16x2(r.x, r.y);
+            pk[2 * k + 1] = tc::pack_bf16x2(r.z, r.w);
+          }
 #pragma unroll
-            for (int k = 0; k < 32; ++k)
-              if (k < ncol) o[k] = v[k] * g.scale;
+          for (int k = 0; k < 4; ++k)
+            *reinterpret_cast<uint4*>(rout2 + ((k ^ ((lane >> 1) & 3)) << 4)) =
+                make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+        }
+        tc::fence_proxy_async_smem();           // generic writes -> async-proxy reads
+        __syncwarp();
+        if (lane == 0) {
+          // (a box wholly past the last row or column stores nothing: skip it)
+          if (row0 < g.rows && n0 + ci * 32 < g.cols) {
+            tc::tma_store_3d(&tmO, sbuf, n0 + ci * 32, row0, bz);
+            if (EPI == EPI_RESIDUAL) tc::tma_store_3d(&tmO2, sbuf + ES::OUT2_OFF, n0 + ci * 32, row0, bz);
+          }
+          tc::bulk_commit();
+          if (EPI == EPI_RESIDUAL && ci + 2 < NCH) {
+            // this buffer's residual input is consumed: fetch the chunk after next
+            tc::mbar_arrive_expect_tx(&res_bar[q][bb], 4096);
+            tc::tma_load_3d(&tmO, &res_bar[q][bb], sbuf + ES::RES_OFF, n0 + 32 * (ci + 2), row0, bz);
+            res_pend |= 1u << bb;
           }
         }
       }
       tc::tc_fence_before();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&tempty_bar[b]);
+      if (!ok) s_abort = 1;
+    }
+    // stores must be complete and residual loads landed before the CTA exits
+    // (a break above can leave prefetched residual chunks in flight)
+    if (lane == 0) {
+      tc::bulk_wait_all();
+      for (int bb = 0; bb < 2; ++bb)
+        if ((res_pend >> bb) & 1u) tc::mbar_wait(&res_bar[q][bb], (res_par >> bb) & 1u, g.status, kErrGemmWait);
     }
   }
   tc::tc_fence_before();
@@ -374,11 +410,30 @@ int num_sms_cached() {
   return n;
 }
 
-template <int BN, int STAGES, int EPI>
-cudaError_t launch_t(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b, const TcArgs& t,
-                     int grid, cudaStream_t s) {
-  auto kern = gemm_tc_kernel<BN, STAGES, EPI>;
-  constexpr int smem = Smem<BN, STAGES>::BYTES;
+// Output tensor [batch][rows][cols] (row stride ld, batch stride sb elements)
+// as 32 x 32 x 1 boxes: fp32 rows of 128 B with the 128-byte swizzle, bf16 rows
+// of 64 B with the 64-byte swizzle (the layouts the epilogue writes).
+bool make_out_map(CUtensorMap* m, void* ptr, bool f32, long long rows, long long cols, long long ld,
+                  long long batch, long long sb) {
+  auto enc = get_encode();
+  if (!enc) return false;
+  const long long es = f32 ? 4 : 2;
+  cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)rows, (cuuint64_t)batch};
+  cuuint64_t strides[2] = {(cuuint64_t)(ld * es), (cuuint64_t)((batch > 1 ? sb : rows * ld) * es)};
+  cuuint32_t box[3] = {32, 32, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, ptr, dims,
+                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int BN, int EPI>
+cudaError_t launch_t(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b, const CUtensorMap& o,
+                     const CUtensorMap& o2, const TcArgs& t, int grid, cudaStream_t s) {
+  auto kern = gemm_tc_kernel<BN, EPI>;
+  constexpr int smem = Smem<BN, EPI>::BYTES;
   static bool attr = false;
   if (!attr) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -395,17 +450,17 @@ cudaError_t launch_t(const CUtensorMap& a0, const CUtensorMap& a1, const CUtenso
   la[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = la;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, a0, a1, b, t);
+  return cudaLaunchKernelEx(&cfg, kern, a0, a1, b, o, o2, t);
 }
 
-template <int BN, int STAGES>
+template <int BN>
 cudaError_t launch_epi(int epi, const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b,
-                       const TcArgs& t, int grid, cudaStream_t s) {
+                       const CUtensorMap& o, const CUtensorMap& o2, const TcArgs& t, int grid, cudaStream_t s) {
   switch (epi) {
-    case EPI_BIAS: return launch_t<BN, STAGES, EPI_BIAS>(a0, a1, b, t, grid, s);
-    case EPI_BIAS_RELU: return launch_t<BN, STAGES, EPI_BIAS_RELU>(a0, a1, b, t, grid, s);
-    case EPI_RESIDUAL: return launch_t<BN, STAGES, EPI_RESIDUAL>(a0, a1, b, t, grid, s);
-    default: return launch_t<BN, STAGES, EPI_SCALE>(a0, a1, b, t, grid, s);
+    case EPI_BIAS: return launch_t<BN, EPI_BIAS>(a0, a1, b, o, o2, t, grid, s);
+    case EPI_BIAS_RELU: return launch_t<BN, EPI_BIAS_RELU>(a0, a1, b, o, o2, t, grid, s);
+    case EPI_RESIDUAL: return launch_t<BN, EPI_RESIDUAL>(a0, a1, b, o, o2, t, grid, s);
+    default: return launch_t<BN, EPI_SCALE>(a0, a1, b, o, o2, t, grid, s);
   }
 }
 
@@ -418,8 +473,13 @@ bool tc_available() { return get_encode() != nullptr; }
 cudaError_t launch_gemm_tc(const GemmArgs& g, int epi, int batch, cudaStream_t s, unsigned* status) {
   if (g.rows <= 0 || g.cols <= 0 || batch <= 0) return cudaSuccess;
   if (g.K % BK || g.k_split % BK || g.lda % 8) return cudaErrorInvalidValue;
+  // the output tensor maps need 16-byte row (and batch) strides
+  const int align_elems = (epi == EPI_BIAS || epi == EPI_BIAS_RELU) ? 8 : 4;
+  if (g.ldo % align_elems || (epi == EPI_RESIDUAL && g.ldo % 8)) return cudaErrorInvalidValue;
+  if (batch > 1 && g.strideO % align_elems) return cudaErrorInvalidValue;
   // Column tile: fewest waves of (tile work + a fixed per-tile latency) over the
-  // SMs; among ties the wider tile (A is read fewer times).
+  // SMs; among ties the wider tile (A is read fewer times).  The residual
+  // epilogue needs more staging, which leaves a 256-wide tile too few ring stages.
   const int nsm = num_sms_cached();
   const long long row_tiles = (long long)((g.rows + BM - 1) / BM) * batch;
   int BN = 64;
@@ -428,6 +488,7 @@ cudaError_t launch_gemm_tc(const GemmArgs& g, int epi, int batch, cudaStream_t s
   for (int ci = 0; ci < 4; ++ci) {
     const int bn = cands[ci];
     if (bn != 64 && g.cols % bn != 0) continue;
+    if (epi == EPI_RESIDUAL && bn > 128) continue;
     const long long tiles = row_tiles * ((g.cols + bn - 1) / bn);
     const double waves = std::ceil((double)tiles / nsm);
     const double cost = waves * (bn + 64.0);
@@ -455,13 +516,22 @@ cudaError_t launch_gemm_tc(const GemmArgs& g, int epi, int batch, cudaStream_t s
   t.b_row0 = 0;
   t.bias = g.bias; t.out = g.out; t.out2 = g.out2; t.ldo = g.ldo; t.strideO = g.strideO;
   t.scale = g.scale; t.status = status;
+  // outputs: bf16 (bias epilogues), fp32 scores, fp32 residual stream + its bf16 copy
+  CUtensorMap o, o2;
+  const bool f32 = epi == EPI_SCALE || epi == EPI_RESIDUAL;
+  if (!make_out_map(&o, g.out, f32, g.rows, g.cols, g.ldo, batch, g.strideO)) return cudaErrorInvalidValue;
+  if (epi == EPI_RESIDUAL) {
+    if (!make_out_map(&o2, g.out2, false, g.rows, g.cols, g.ldo, batch, g.strideO)) return cudaErrorInvalidValue;
+  } else {
+    o2 = o;
+  }
   const long long tiles = row_tiles * ((g.cols + BN - 1) / BN);
   const int grid = (int)(tiles < nsm ? tiles : nsm);
   switch (BN) {
-    case 256: return launch_epi<256, 3>(epi, a0, a1, b, t, grid, s);
-    case 192: return launch_epi<192, 4>(epi, a0, a1, b, t, grid, s);
-    case 128: return launch_epi<128, 4>(epi, a0, a1, b, t, grid, s);
-    default: return launch_epi<64, 6>(epi, a0, a1, b, t, grid, s);
+    case 256: return launch_epi<256>(epi, a0, a1, b, o, o2, t, grid, s);
+    case 192: return launch_epi<192>(epi, a0, a1, b, o, o2, t, grid, s);
+    case 128: return launch_epi<128>(epi, a0, a1, b, o, o2, t, grid, s);
+    default: return launch_epi<64>(epi, a0, a1, b, o, o2, t, grid, s);
   }
 }
 

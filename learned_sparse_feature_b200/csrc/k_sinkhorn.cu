@@ -299,9 +299,13 @@ __global__ void __launch_bounds__(256 * SPLIT, 1) sinkhorn_kernel(SinkhornArgs a
 #pragma unroll
       for (int c = 0; c < CPW; ++c) colacc[c] = 0.f;
       float colbin = 0.f;
-      const float4* v4 = reinterpret_cast<const float4*>(vbuf);   // read in the loop: saves registers
+      const float4* v4 = reinterpret_cast<const float4*>(vbuf);
       const float vb = vbuf[LDW];
       const int g0 = part * NQW;                  // this warp's first float4 group
+      // this lane's column potentials, re-read from shared memory per row (held
+      // in registers next to the row and its column sums they cost more in
+      // lost latency hiding than the shared-memory reads)
+      auto vq_at = [&](int qq) -> float4 { return v4[(g0 + qq) * 32 + lane]; };
       const bool bin_lane = part == 0 && lane == 0;
       int k = 0;                                  // rows taken by the team (slot parity)
       for (int r = r0 + team; r < r1; r += NTEAM, ++k) {
@@ -316,7 +320,7 @@ __global__ void __launch_bounds__(256 * SPLIT, 1) sinkhorn_kernel(SinkhornArgs a
             float mx = bin_lane ? alpha2 + vb : -INFINITY;
 #pragma unroll
             for (int qq = 0; qq < NQW; ++qq) {
-              const float4 vq = v4[(g0 + qq) * 32 + lane];
+              const float4 vq = vq_at(qq);
               mx = fmaxf(mx, fmaxf(fmaxf(e[4 * qq] + vq.x, e[4 * qq + 1] + vq.y),
                                    fmaxf(e[4 * qq + 2] + vq.z, e[4 * qq + 3] + vq.w)));
             }
@@ -332,7 +336,7 @@ __global__ void __launch_bounds__(256 * SPLIT, 1) sinkhorn_kernel(SinkhornArgs a
           float part_s = 0.f;
 #pragma unroll
           for (int qq = 0; qq < NQW; ++qq) {
-            const float4 vq = v4[(g0 + qq) * 32 + lane];
+            const float4 vq = vq_at(qq);
             const float x0 = ex2((e[4 * qq] + vq.x) - m);
             const float x1 = ex2((e[4 * qq + 1] + vq.y) - m);
             const float x2 = ex2((e[4 * qq + 2] + vq.z) - m);
@@ -366,65 +370,82 @@ __global__ void __launch_bounds__(256 * SPLIT, 1) sinkhorn_kernel(SinkhornArgs a
       // CTA column sums: a 3-round tree over the teams through shared memory
       // (8 -> 4 -> 2 -> 1 partial vectors; the parts of a team own disjoint
       // columns of the same vectors; shared fp32 atomics from 8 warps on the
-      // same addresses are an order of magnitude slower)
+      // same addresses are an order of magnitude slower).  Each round writes
+      // into slots that only the writing team itself read in the round before,
+      // so one barrier per round suffices:
+      //   round 1: teams 4-7 -> slots 0-3, read by teams 0-3;
+      //   round 2: teams 2-3 -> slots 2-3, read by teams 0-1;
+      //   round 3: team 1    -> slot 1,    read by team 0, which writes the total.
+      auto put = [&](int slot) {
+        float4* dst = reinterpret_cast<float4*>(xbuf + (size_t)slot * CV);
 #pragma unroll
-      for (int half = NTEAM / 2; half >= 1; half >>= 1) {
-        if (team >= half && team < 2 * half) {
-          float4* dst = reinterpret_cast<float4*>(xbuf + (size_t)(team - half) * CV);
+        for (int qq = 0; qq < NQW; ++qq)
+          dst[(g0 + qq) * 32 + lane] =
+              make_float4(colacc[4 * qq], colacc[4 * qq + 1], colacc[4 * qq + 2], colacc[4 * qq + 3]);
+        if (bin_lane) xbuf[(size_t)slot * CV + LDW] = colbin;
+      };
+      auto take = [&](int slot) {
+        const float4* src = reinterpret_cast<const float4*>(xbuf + (size_t)slot * CV);
 #pragma unroll
-          for (int qq = 0; qq < NQW; ++qq)
-            dst[(g0 + qq) * 32 + lane] =
-                make_float4(colacc[4 * qq], colacc[4 * qq + 1], colacc[4 * qq + 2], colacc[4 * qq + 3]);
-          if (bin_lane) xbuf[(size_t)(team - half) * CV + LDW] = colbin;
+        for (int qq = 0; qq < NQW; ++qq) {
+          const float4 t = src[(g0 + qq) * 32 + lane];
+          colacc[4 * qq] += t.x; colacc[4 * qq + 1] += t.y; colacc[4 * qq + 2] += t.z; colacc[4 * qq + 3] += t.w;
         }
-        __syncthreads();
-        if (team < half) {
-          const float4* src = reinterpret_cast<const float4*>(xbuf + (size_t)team * CV);
-#pragma unroll
-          for (int qq = 0; qq < NQW; ++qq) {
-            const float4 t = src[(g0 + qq) * 32 + lane];
-            colacc[4 * qq] += t.x; colacc[4 * qq + 1] += t.y; colacc[4 * qq + 2] += t.z; colacc[4 * qq + 3] += t.w;
-          }
-          if (bin_lane) colbin += xbuf[(size_t)team * CV + LDW];
-        }
-        __syncthreads();
-      }
+        if (bin_lane) colbin += xbuf[(size_t)slot * CV + LDW];
+      };
+      static_assert(NTEAM == 8, "tree shape");
+      if (team >= 4) put(team - 4);
+      __syncthreads();
+      if (team < 4) take(team);
+      if (team == 2 || team == 3) put(team);
+      __syncthreads();
+      if (team < 2) take(team + 2);
+      if (team == 1) put(1);
+      __syncthreads();
       if (team == 0) {
+        take(1);
         float4* dst = reinterpret_cast<float4*>(ctot);
 #pragma unroll
         for (int qq = 0; qq < NQW; ++qq)
           dst[(g0 + qq) * 32 + lane] =
               make_float4(colacc[4 * qq], colacc[4 * qq + 1], colacc[4 * qq + 2], colacc[4 * qq + 3]);
         if (bin_lane) ctot[LDW] = colbin;
+        if (cpp > 1) fence_proxy_async_smem();    // ctot is the source of a bulk copy
       }
       __syncthreads();
       // ------------------------------------------------ column pass (group)
+      // column totals: ctot (one CTA per pair) or the group's accumulator
+      const float* tot = ctot;
       if (cpp > 1) {
         float* acc_now = acc + (size_t)(it % 3) * Cp;
         float* acc_zero = acc + (size_t)((it + 1) % 3) * Cp;   // last read two barriers ago
-        fence_proxy_async_smem();
-        __syncthreads();
         if (tid == 0) bulk_add_f32(acc_now, ctot, (unsigned)(CV * sizeof(float)));
         for (int j = rank * NT + tid; j < Cp; j += cpp * NT) acc_zero[j] = 0.f;
         if (barrier()) { failed = true; break; }
-        for (int j = tid * 4; j < CV; j += NT * 4)
-          *reinterpret_cast<float4*>(ctot + j) = __ldcg(reinterpret_cast<const float4*>(acc_now + j));
-        __syncthreads();
+        tot = acc_now;
       }
-      // column update (each thread its columns of the shared v), with the guard
+      // column update straight from the totals (each thread its columns of the
+      // shared v), with the guard; a tiny total anywhere sends the whole group
+      // to the exact recomputation below, which rebuilds v from scratch
       bool bad = false;
-      for (int j = tid; j < CV; j += NT) {
-        if (j < N || j == LDW) {
-          const float cm = ctot[j];
-          if (!(cm >= kColTiny && cm < INFINITY)) bad = true;
+      for (int j4 = tid; j4 < CV / 4; j4 += NT) {   // one float4 per thread: one round of latency
+        const float4 c4 = cpp > 1 ? __ldcg(reinterpret_cast<const float4*>(tot) + j4)
+                                  : reinterpret_cast<const float4*>(tot)[j4];
+        float4 v = reinterpret_cast<float4*>(vbuf)[j4];
+        const float cm[4] = {c4.x, c4.y, c4.z, c4.w};
+        float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int j = 4 * j4 + i;
+          if (j < N || j == LDW) {
+            if (!(cm[i] >= kColTiny && cm[i] < INFINITY)) bad = true;
+            else vv[i] += (j < N ? lnu_r2 : lnu_b2) - lg2(cm[i]);
+          }
         }
+        reinterpret_cast<float4*>(vbuf)[j4] = make_float4(vv[0], vv[1], vv[2], vv[3]);
       }
       if (!__syncthreads_or(bad)) {
-        for (int j = tid; j < CV; j += NT) {
-          if (j < N) vbuf[j] += lnu_r2 - lg2(ctot[j]);
-          else if (j == LDW) vbuf[j] += lnu_b2 - lg2(ctot[j]);
-          ctot[j] = 0.f;
-        }
+        // nothing more: the next row pass reads the new v
       } else {
         // exact column LSE: the true column max, then the shifted sum, each
         // combined over the CTA with shared atomics and over the group with
@@ -629,15 +650,36 @@ cudaError_t launch_t(SinkhornArgs a, int num_sms, cudaStream_t s, int* launches)
     const int groups = G / cpp;
     const int conc = a.B < groups ? a.B : groups;
     const double rounds = std::ceil((double)a.B / groups);
-    const double mufu = (double)band * LDW / 16.0 / clk;
-    const double issue = (double)band * (LDW / 32.0 * 6.0 + 60.0) / (4.0 * clk);
-    const double stream_bw = (double)conc * pair_bytes < 100e6 ? 100e9 : 6.5e12 / G;
+    // rows are taken by NTEAM teams in rounds: the busiest team sets the pace
+    const double rows = std::ceil((double)band / NTEAM) * NTEAM;
+    // per row: one MUFU ex2 per element (16 per clock and SM) and the row plus
+    // the column potentials out of shared memory (8 bytes per element at 128
+    // bytes per clock), which overlap poorly
+    const double mufu = rows * LDW * (1.0 / 16.0 + 8.0 / 128.0) / clk;
+    const double issue = rows * (LDW / 32.0 * 6.0 + 60.0) / (4.0 * clk);
+    // rows that are not cached are re-read every iteration by latency-bound
+    // loads: measured about 40 GB/s per SM from L2 and 17 GB/s per SM when the
+    // concurrently processed pairs overflow L2; that time adds to the compute
+    const double stream_bw = (double)conc * pair_bytes < 100e6 ? 40e9 : 17e9;
     const double stream = (double)(band - cached) * LDW * 4 / stream_bw;
     const double sync = cpp == 1 ? 0.2e-6 : 2.5e-6 + cpp * 1.0e-8;
-    double work = mufu > issue ? mufu : issue;
-    work = work > stream ? work : stream;
+    const double work = (mufu > issue ? mufu : issue) + stream;
     const double t = rounds * (work + sync);
     if (t < best_t) { best_t = t; best_cpp = cpp; best_cached = cached; best_band = band; }
+  }
+  if (const char* f = std::getenv("SG_SINKHORN_CPP")) {
+    // tuning override of the CTAs per pair (ignored when it does not fit)
+    const int cpp = std::atoi(f);
+    if (cpp >= 1 && cpp <= G && cpp <= R) {
+      const int band = (R + cpp - 1) / cpp;
+      const size_t ubytes = (size_t)((band + 3) & ~3) * 4;
+      if (fixed + ubytes <= kMaxSmem) {
+        const int fit = (int)((kMaxSmem - fixed - ubytes) / ((size_t)LDW * 4));
+        best_cpp = cpp;
+        best_band = band;
+        best_cached = band < fit ? band : fit;
+      }
+    }
   }
   if (best_cpp == 0) return cudaErrorInvalidConfiguration;
   a.cpp = best_cpp;

@@ -574,7 +574,17 @@ sg_status_t sg_scores(sg_handle* h, int B, int M, int N, const float* kpts0, con
   cudaStream_t s = (cudaStream_t)stream;
   Inputs in{kpts0, conf0, desc0, kpts1, conf1, desc1};
   int launches = 0;
-  return cuda_err(h, run_network(h, B, M, N, in, out_scores, N, (long long)M * N, s, &launches));
+  // The tensor-core score GEMM stores 16-byte-aligned rows: a caller layout
+  // that is not (N % 4 != 0 or a misaligned buffer) goes through the handle's
+  // score buffer and one strided copy.
+  const bool direct = !h->use_tc || (N % 4 == 0 && (reinterpret_cast<uintptr_t>(out_scores) & 15) == 0);
+  if (direct) return cuda_err(h, run_network(h, B, M, N, in, out_scores, N, (long long)M * N, s, &launches));
+  const long long lds = (N + 3) & ~3;
+  cudaError_t e = run_network(h, B, M, N, in, h->Z, lds, (long long)M * lds, s, &launches);
+  if (e == cudaSuccess)
+    e = cudaMemcpy2DAsync(out_scores, (size_t)N * sizeof(float), h->Z, (size_t)lds * sizeof(float),
+                          (size_t)N * sizeof(float), (size_t)B * M, cudaMemcpyDeviceToDevice, s);
+  return cuda_err(h, e);
 }
 
 sg_status_t sg_optimal_transport(sg_handle* h, int B, int M, int N, const float* scores,
