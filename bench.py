@@ -56,6 +56,37 @@ def whole_job_rate(pairs_per_rank: int, world: int, steps: int, total_ms_max: fl
     return pairs_per_rank * world * steps / (total_ms_max / 1000.0)
 
 
+# kernel class -> (profile summary stem, kernel source) for the measured DRAM traffic
+TRAFFIC_PROFILES = {
+    "sinkhorn": ("sinkhorn", "learned_sparse_feature_b200/csrc/k_sinkhorn.cu"),
+    "attention": ("attention", "learned_sparse_feature_b200/csrc/k_attn_tc.cu"),
+}
+
+
+def measured_traffic(kernel_class: str, workload: str):
+    """DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from the
+    committed ncu summary of this kernel and workload, or None when there is no
+    summary or the kernel source changed since it was captured (the summary
+    records the source's SHA-256)."""
+    import hashlib
+    import re
+
+    if kernel_class not in TRAFFIC_PROFILES:
+        return None, None
+    stem, src = TRAFFIC_PROFILES[kernel_class]
+    path = os.path.join(ROOT, "profiles", f"{stem}_{workload}.md")
+    try:
+        text = open(path).read()
+        digest = hashlib.sha256(open(os.path.join(ROOT, src), "rb").read()).hexdigest()
+    except OSError:
+        return None, None
+    m_sha = re.search(r"^source_sha256: ([0-9a-f]{64})", text, re.M)
+    m_tr = re.search(r"^traffic_bytes_per_launch: (\d+)", text, re.M)
+    if not m_sha or not m_tr or m_sha.group(1) != digest:
+        return None, os.path.relpath(path, ROOT)
+    return int(m_tr.group(1)), os.path.relpath(path, ROOT)
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -84,7 +115,7 @@ def algorithmic_work(B, M, N, n_stages=18, T=100, D=256):
         "mlp2_gemm": ("tensor", 2.0 * R * D * (2 * D)),
         "proj_gemm": ("tensor", 2.0 * R * D * D),
         "score_gemm": ("tensor", 2.0 * B * M * N * D),
-        # the spec model of Sinkhorn traffic: 2 passes over E fp32 per iteration
+        # streamed-byte model of the transport: two fp32 passes over the augmented matrix per iteration
         "sinkhorn": ("hbm", 2.0 * T * 4 * E * B),
     }
 
@@ -336,9 +367,22 @@ def run_native(args, w):
         achieved, peak, unit = units / avg_s / 1e12, peaks["bf16_tflops"], "TFLOP/s"
     else:
         achieved, peak, unit = units / avg_s / 1e12, None, "TFLOP/s"
+    traffic, traffic_src = measured_traffic(dom, w.name)
     roofline = {"bound": bound, "kernel": dom, "achieved": achieved, "peak": peak, "unit": unit,
-                "frac": (achieved / peak) if peak else None, "traffic": None,
+                "frac": (achieved / peak) if peak else None, "traffic": traffic,
+                "traffic_source": traffic_src,
                 "peak_source": peak_src + (" (burst)" if bound == "tensor" else "")}
+    if dom == "sinkhorn":
+        # the other bounds of the transport kernel: one ex2 per element and
+        # iteration on the MUFU (16 per clock and SM), and the compulsory bytes
+        # (read S, write log P: 8 E)
+        E = (M + 1) * (N + 1) * B
+        sm_clock = (clk.get("sm_mhz") or 1965.0) * 1e6
+        roofline["other_bounds_ms"] = {
+            "mufu_ex2": 100 * E / (148 * 16 * sm_clock) * 1e3,
+            "compulsory_bytes": 8 * E / (peaks["hbm_gbs"] * 1e9) * 1e3,
+            "kernel": avg_s * 1e3,
+        }
     breakdown = {}
     for k, (ms, n) in per_class.items():
         if n == 0:

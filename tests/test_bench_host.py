@@ -1,0 +1,50 @@
+"""Host logic of bench.py that needs no GPU: the measured-traffic lookup, which
+must go stale (None) as soon as the kernel source differs from the one the
+ncu summary was captured on, and the algorithmic-work model."""
+import hashlib
+import os
+
+import bench
+
+
+def _tree(tmp_path, src_text, recorded_sha, traffic=12345):
+    (tmp_path / "profiles").mkdir()
+    src = tmp_path / "learned_sparse_feature_b200" / "csrc"
+    src.mkdir(parents=True)
+    (src / "k_sinkhorn.cu").write_text(src_text)
+    (tmp_path / "profiles" / "sinkhorn_pair2048.md").write_text(
+        f"# summary\n\nsource_sha256: {recorded_sha} (k_sinkhorn.cu)\ntraffic_bytes_per_launch: {traffic}\n")
+
+
+def test_traffic_is_read_when_the_source_matches(tmp_path, monkeypatch):
+    text = "kernel v1"
+    _tree(tmp_path, text, hashlib.sha256(text.encode()).hexdigest())
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    traffic, src = bench.measured_traffic("sinkhorn", "pair2048")
+    assert traffic == 12345
+    assert src == os.path.join("profiles", "sinkhorn_pair2048.md")
+
+
+def test_traffic_goes_stale_when_the_kernel_changes(tmp_path, monkeypatch):
+    _tree(tmp_path, "kernel v2", hashlib.sha256(b"kernel v1").hexdigest())
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    traffic, _ = bench.measured_traffic("sinkhorn", "pair2048")
+    assert traffic is None
+
+
+def test_traffic_absent_for_other_kernels_and_workloads(tmp_path, monkeypatch):
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.measured_traffic("qkv_gemm", "pair2048") == (None, None)
+    assert bench.measured_traffic("sinkhorn", "pair512") == (None, None)
+
+
+def test_algorithmic_work_matches_the_pages_counts():
+    # pair2048: the attention FLOPs of 18 stages and the streamed-byte model of
+    # 100 Sinkhorn iterations (two fp32 passes over the augmented matrix each)
+    w = bench.algorithmic_work(1, 2048, 2048)
+    bound, flops = w["attention"]
+    assert bound == "tensor"
+    assert abs(flops * 18 - 36 * 256 * 4096 ** 2) / (36 * 256 * 4096 ** 2) < 1e-12
+    bound, bytes_ = w["sinkhorn"]
+    assert bound == "hbm"
+    assert bytes_ == 2 * 100 * 4 * 2049 * 2049
