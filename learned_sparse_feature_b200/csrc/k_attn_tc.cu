@@ -287,7 +287,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm, AttnTcArgs a) {
         tc::tmem_ld32_async(t_s + 32, s1);
         tc::tmem_ld32_async(t_s + 64, s2);
         tc::tmem_ld32_async(t_s + 96, s3);
-        tc::tmem_wait_ld();
+        tc::tmem_wait_ld(s0);                       // (one wait covers all four loads; the
+        tc::tmem_wait_ld(s1);                       //  others only pin their registers)
+        tc::tmem_wait_ld(s2);
+        tc::tmem_wait_ld(s3);
       }
       const int valid = nk - j * KT;                 // keys of this tile that exist
       if (valid < KT) {

@@ -272,12 +272,16 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
       tc::tc_fence_after();
       const uint32_t trow = tmem + b * BNA + ((uint32_t)(q * 32) << 16);
       bool ok = true;
-#pragma unroll 1
+      // chunk ci's accumulator columns arrive while chunk ci - 1 is processed
+      float va[32], vb[32];
+      tc::tmem_ld32_async(trow, va);            // warp-collective: every lane takes part
+#pragma unroll
       for (int ci = 0; ci < NCH; ++ci, ++chunk) {
         const int bb = chunk & 1;
         uint8_t* sbuf = wbuf + bb * ES::BUF;
-        float v[32];
-        tc::tmem_ld32(trow + ci * 32, v);       // warp-collective: every lane takes part
+        float (&v)[32] = (ci & 1) ? vb : va;
+        tc::tmem_wait_ld(v);
+        if (ci + 1 < NCH) tc::tmem_ld32_async(trow + (ci + 1) * 32, (ci & 1) ? va : vb);
         // the store issued from this buffer two chunks ago must have read it
         if (lane == 0) tc::bulk_wait_read<1>();
         __syncwarp();
