@@ -126,6 +126,13 @@ def make_weights(seed: int = 0, n_stages: int = N_STAGES, d: int = D,
     w["Wf"] = _kaiming_uniform(rng, d, d, gain_final_proj)
     w["bf"] = _bias(rng, d, d)
     w["bin_score"] = np.float32(BIN_SCORE)
+    # double-softmax matching head (projection and matchability), from a stream
+    # of its own so that the weights above do not depend on it
+    rng_h = np.random.default_rng([seed, 1])
+    w["lg_Wp"] = _kaiming_uniform(rng_h, d, d, gain_final_proj)
+    w["lg_bp"] = _bias(rng_h, d, d)
+    w["lg_wz"] = _kaiming_uniform(rng_h, 1, d, gain_final_proj)[0]
+    w["lg_bz"] = np.float32(_bias(rng_h, 1, d)[0])
     return w
 
 

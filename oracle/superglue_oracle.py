@@ -253,13 +253,64 @@ def extract_matches(logP, threshold):
     return matches0, matches1, mscores0, mscores1
 
 
+# --------------------------------------------------------------------------- double-softmax head
+def log_sigmoid(x):
+    """log(1 / (1 + exp(-x))) = min(x, 0) - log(1 + exp(-|x|)) (stable form)."""
+    x = _as64(x)
+    return np.minimum(x, 0.0) - np.log1p(np.exp(-np.abs(x)))
+
+
+def log_softmax(x, axis):
+    """x - log sum exp along `axis`."""
+    x = _as64(x)
+    return x - np.expand_dims(logsumexp(x, axis), axis)
+
+
+def double_softmax_log_assignment(sim, z0, z1):
+    """The matching head that replaces the dustbin and Sinkhorn ("论文解读:LightGlue,
+    让稀疏特征匹配随难度自适应地快" (LightGlue review), section 2.4 匹配头, the
+    sigmoid_log_double_softmax listing): an (M+1) x (N+1) log assignment whose real
+    block is log_softmax over j (each row) + log_softmax over i (each column) +
+    log sigmoid(z0_i) + log sigmoid(z1_j); the last column is log sigmoid(-z0_i),
+    the last row log sigmoid(-z1_j), the corner 0.
+    Pinned by: torch log_softmax / logsigmoid in float64, a 2 x 2 closed form, the
+    dustbin complement exp(last column) = 1 - sigmoid(z0), planted mistakes."""
+    sim = _as64(sim)
+    z0, z1 = _as64(z0), _as64(z1)
+    M, N = sim.shape
+    out = np.zeros((M + 1, N + 1), F64)
+    out[:M, :N] = (log_softmax(sim, 1) + log_softmax(sim, 0)
+                   + log_sigmoid(z0)[:, None] + log_sigmoid(z1)[None, :])
+    out[:M, N] = log_sigmoid(-z0)
+    out[M, :N] = log_sigmoid(-z1)
+    return out
+
+
+def double_softmax_head(x0, x1, Wp, bp, wz, bz):
+    """Similarity and matchability of the double-softmax head (LightGlue review,
+    section 2.4, MatchAssignment.forward): m = final_proj(x) / D^(1/4) for both
+    images, sim_ij = <m0_i, m1_j>; z = matchability(x) = x . wz + bz on the GNN
+    states themselves (not on m).  Returns (log assignment, sim, z0, z1).
+    Pinned by: the torch MatchAssignment composition in float64."""
+    x0, x1 = _as64(x0), _as64(x1)
+    d = x0.shape[1]
+    m0 = linear(x0, Wp, bp) / d ** 0.25
+    m1 = linear(x1, Wp, bp) / d ** 0.25
+    sim = m0 @ m1.T
+    z0 = x0 @ _as64(wz) + float(bz)
+    z1 = x1 @ _as64(wz) + float(bz)
+    return double_softmax_log_assignment(sim, z0, z1), sim, z0, z1
+
+
 # --------------------------------------------------------------------------- whole pass
 def superglue_pair(kpts0, conf0, desc0, kpts1, conf1, desc1, weights,
                    img_w=640.0, img_h=480.0, heads=4, iters=100,
-                   threshold=0.2, eps=1e-5, norm_mode=0, n_stages=None):
+                   threshold=0.2, eps=1e-5, norm_mode=0, n_stages=None, head="sinkhorn"):
     """One pair through the whole matcher.  Inputs point-major: kpts (n, 2) px,
     conf (n,), desc (n, D).  Returns a dict with log_P ((M+1) x (N+1)),
-    matches0/1, mscores0/1.
+    matches0/1, mscores0/1.  head="double_softmax" replaces the score matrix,
+    dustbin and Sinkhorn by the double-softmax head on the same GNN states
+    (extraction unchanged; LightGlue's default threshold is 0.1).
 
     Empty input (M == 0 or N == 0): matches -1 and scores 0, no log_P
     [Jazihars notes, forward(), the "no keypoints" early return]."""
@@ -273,6 +324,12 @@ def superglue_pair(kpts0, conf0, desc0, kpts1, conf1, desc1, weights,
     x0 = keypoint_encoder(k0, conf0, desc0, weights, eps)
     x1 = keypoint_encoder(k1, conf1, desc1, weights, eps)
     x0, x1 = attentional_gnn(x0, x1, weights, heads, eps, n_stages)
+    if head == "double_softmax":
+        logP, sim, z0, z1 = double_softmax_head(x0, x1, weights["lg_Wp"], weights["lg_bp"],
+                                                weights["lg_wz"], weights["lg_bz"])
+        m0, m1, s0, s1 = extract_matches(logP, threshold)
+        return {"log_P": logP, "matches0": m0, "matches1": m1, "mscores0": s0, "mscores1": s1,
+                "scores": sim, "z0": z0, "z1": z1}
     S = score_matrix(x0, x1, weights["Wf"], weights["bf"])
     logP = log_optimal_transport(S, float(weights["bin_score"]), iters)
     m0, m1, s0, s1 = extract_matches(logP, threshold)

@@ -31,6 +31,11 @@ PIN_TESTS = [
     (pins.test_extraction_hand_built, False),
     (pins.test_extraction_ties_take_lowest_index_and_threshold_is_strict, False),
     (pins.test_score_matrix_scale_matches_library_attention, True),
+    (pins.test_double_softmax_matches_torch_log_softmax_and_logsigmoid, False),
+    (pins.test_double_softmax_two_by_two_closed_form, False),
+    (pins.test_log_sigmoid_is_stable_and_complements, False),
+    (pins.test_double_softmax_head_matches_torch_modules, True),
+    (pins.test_double_softmax_recovers_a_planted_permutation, False),
 ]
 
 
@@ -178,7 +183,66 @@ def _prop_message_first(x, src, st, heads, eps):
     return O.mlp(z, [st["W1"], st["W2"]], [st["b1"], st["b2"]], [st["bn1"]], eps)
 
 
+_dsm_assign = O.double_softmax_log_assignment
+
+
+def _dsm_same_axis_twice(sim, z0, z1):
+    out = _dsm_assign(sim, z0, z1)
+    M, N = np.shape(sim)
+    out[:M, :N] += O.log_softmax(sim, 1) - O.log_softmax(sim, 0)
+    return out
+
+
+def _dsm_no_certainty(sim, z0, z1):
+    out = _dsm_assign(sim, z0, z1)
+    M, N = np.shape(sim)
+    out[:M, :N] -= O.log_sigmoid(z0)[:, None] + O.log_sigmoid(z1)[None, :]
+    return out
+
+
+def _dsm_dustbin_sign(sim, z0, z1):
+    out = _dsm_assign(sim, z0, z1)
+    M, N = np.shape(sim)
+    out[:M, N] = O.log_sigmoid(z0)
+    out[M, :N] = O.log_sigmoid(z1)
+    return out
+
+
+def _dsm_corner_one(sim, z0, z1):
+    out = _dsm_assign(sim, z0, z1)
+    out[-1, -1] = 1.0
+    return out
+
+
+def _head_sqrt_scale(x0, x1, Wp, bp, wz, bz):
+    x0, x1 = np.asarray(x0, float), np.asarray(x1, float)
+    d = x0.shape[1]
+    m0 = O.linear(x0, Wp, bp) / d ** 0.5
+    m1 = O.linear(x1, Wp, bp) / d ** 0.5
+    sim = m0 @ m1.T
+    z0 = x0 @ np.asarray(wz, float) + float(bz)
+    z1 = x1 @ np.asarray(wz, float) + float(bz)
+    return O.double_softmax_log_assignment(sim, z0, z1), sim, z0, z1
+
+
+def _head_matchability_on_projection(x0, x1, Wp, bp, wz, bz):
+    x0, x1 = np.asarray(x0, float), np.asarray(x1, float)
+    d = x0.shape[1]
+    m0 = O.linear(x0, Wp, bp) / d ** 0.25
+    m1 = O.linear(x1, Wp, bp) / d ** 0.25
+    sim = m0 @ m1.T
+    z0 = m0 @ np.asarray(wz, float) + float(bz)
+    z1 = m1 @ np.asarray(wz, float) + float(bz)
+    return O.double_softmax_log_assignment(sim, z0, z1), sim, z0, z1
+
+
 MUTATIONS = {
+    "double softmax over one axis twice": ("double_softmax_log_assignment", _dsm_same_axis_twice),
+    "double softmax without certainties": ("double_softmax_log_assignment", _dsm_no_certainty),
+    "double softmax dustbin sign": ("double_softmax_log_assignment", _dsm_dustbin_sign),
+    "double softmax corner not zero": ("double_softmax_log_assignment", _dsm_corner_one),
+    "head scaled by D^(1/2)": ("double_softmax_head", _head_sqrt_scale),
+    "matchability on the projection": ("double_softmax_head", _head_matchability_on_projection),
     "attention scale 1/sqrt(D)": ("attend", _attend_wrong_scale),
     "softmax over queries": ("attend", _attend_wrong_axis),
     "BN eps outside sqrt": ("batchnorm_eval", _bn_eps_outside),

@@ -369,3 +369,88 @@ def test_score_matrix_scale_matches_library_attention(weights):
     ref = torch.nn.functional.scaled_dot_product_attention(
         torch.tensor(f0[None]), torch.tensor(f1[None]), torch.eye(9, dtype=torch.float64)[None])[0]
     np.testing.assert_allclose(O.softmax(S, axis=1), ref.numpy(), rtol=1e-10, atol=1e-13)
+
+
+# --------------------------------------------------------------------------- double-softmax head
+def _dsm_inputs(seed=3, M=5, N=4):
+    rng = np.random.default_rng(seed)
+    return rng.normal(0, 2.0, (M, N)), rng.normal(0, 1.5, M), rng.normal(0, 1.5, N)
+
+
+def test_double_softmax_matches_torch_log_softmax_and_logsigmoid():
+    import torch.nn.functional as F
+    sim, z0, z1 = _dsm_inputs()
+    M, N = sim.shape
+    got = O.double_softmax_log_assignment(sim, z0, z1)
+    s = torch.from_numpy(sim)
+    a, b = torch.from_numpy(z0), torch.from_numpy(z1)
+    real = F.log_softmax(s, 1) + F.log_softmax(s, 0) + F.logsigmoid(a)[:, None] + F.logsigmoid(b)[None, :]
+    np.testing.assert_allclose(got[:M, :N], real.numpy(), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(got[:M, N], F.logsigmoid(-a).numpy(), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(got[M, :N], F.logsigmoid(-b).numpy(), rtol=0, atol=1e-12)
+    assert got[M, N] == 0.0
+
+
+def test_double_softmax_two_by_two_closed_form():
+    # sim = [[1, 0], [0, 2]], z0 = (0, ln 3), z1 = (ln 2, 0): every entry by hand
+    sim = np.array([[1.0, 0.0], [0.0, 2.0]])
+    z0 = np.array([0.0, math.log(3.0)])
+    z1 = np.array([math.log(2.0), 0.0])
+    e = math.e
+    sig = lambda t: 1.0 / (1.0 + math.exp(-t))
+    row = [[e / (e + 1), 1 / (e + 1)], [1 / (1 + e * e), e * e / (1 + e * e)]]
+    col = [[e / (e + 1), 1 / (1 + e * e)], [1 / (e + 1), e * e / (1 + e * e)]]
+    got = np.exp(O.double_softmax_log_assignment(sim, z0, z1))
+    for i in range(2):
+        for j in range(2):
+            want = row[i][j] * col[i][j] * sig(z0[i]) * sig(z1[j])
+            assert abs(got[i, j] - want) < 1e-14
+    assert abs(got[0, 2] - 0.5) < 1e-15 and abs(got[1, 2] - 0.25) < 1e-15
+    assert abs(got[2, 0] - 1.0 / 3.0) < 1e-15 and abs(got[2, 1] - 0.5) < 1e-15
+    assert got[2, 2] == 1.0
+
+
+def test_log_sigmoid_is_stable_and_complements():
+    x = np.array([-60.0, -5.0, -1e-3, 0.0, 2.0, 60.0])
+    ls = O.log_sigmoid(x)
+    assert np.all(np.isfinite(ls))
+    assert abs(ls[0] - (-60.0 - math.exp(-60.0))) < 1e-12
+    assert abs(ls[-1] + math.exp(-60.0)) < 1e-30
+    np.testing.assert_allclose(np.exp(ls) + np.exp(O.log_sigmoid(-x)), 1.0, rtol=0, atol=1e-15)
+
+
+def test_double_softmax_head_matches_torch_modules(weights):
+    rng = np.random.default_rng(11)
+    x0 = rng.normal(0, 1, (7, synth.D))
+    x1 = rng.normal(0, 1, (6, synth.D))
+    logP, sim, z0, z1 = O.double_softmax_head(x0, x1, weights["lg_Wp"], weights["lg_bp"],
+                                              weights["lg_wz"], weights["lg_bz"])
+    with torch.no_grad():
+        proj = torch.nn.Linear(synth.D, synth.D).double()
+        proj.weight.copy_(torch.from_numpy(np.asarray(weights["lg_Wp"], np.float64)))
+        proj.bias.copy_(torch.from_numpy(np.asarray(weights["lg_bp"], np.float64)))
+        mz = torch.nn.Linear(synth.D, 1).double()
+        mz.weight.copy_(torch.from_numpy(np.asarray(weights["lg_wz"], np.float64))[None, :])
+        mz.bias.fill_(float(weights["lg_bz"]))
+        t0, t1 = torch.from_numpy(x0), torch.from_numpy(x1)
+        m0 = proj(t0) / synth.D ** 0.25
+        m1 = proj(t1) / synth.D ** 0.25
+        want_sim = torch.einsum("md,nd->mn", m0, m1).numpy()
+        want_z0 = mz(t0)[:, 0].numpy()
+        want_z1 = mz(t1)[:, 0].numpy()
+    np.testing.assert_allclose(sim, want_sim, rtol=1e-12, atol=1e-10)
+    np.testing.assert_allclose(z0, want_z0, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(z1, want_z1, rtol=1e-12, atol=1e-12)
+
+
+def test_double_softmax_recovers_a_planted_permutation():
+    # a sharp permutation similarity and confident points: the head's mutual
+    # argmax is the permutation, each with probability near 1
+    perm = np.array([2, 0, 3, 1])
+    sim = np.full((4, 4), -10.0)
+    sim[np.arange(4), perm] = 10.0
+    logP = O.double_softmax_log_assignment(sim, np.full(4, 20.0), np.full(4, 20.0))
+    m0, m1, s0, _ = O.extract_matches(logP, 0.1)
+    np.testing.assert_array_equal(m0, perm)
+    np.testing.assert_array_equal(m1[perm], np.arange(4))
+    assert np.all(s0 > 0.99)
