@@ -61,6 +61,9 @@ def whole_job_rate(pairs_per_rank: int, world: int, steps: int, total_ms_max: fl
 # not stated) = 14.29 pairs/s.  Context, not the target.
 PAGES_PAIRS_PER_S = {"pair2048": 1000.0 / 70.0}
 
+# the double-softmax head's default filter threshold (LightGlue review: filter_threshold=0.1)
+DSM_THRESHOLD = 0.1
+
 # kernel class -> (profile summary stem, kernel source) for the measured DRAM traffic
 TRAFFIC_PROFILES = {
     "sinkhorn": ("sinkhorn", "learned_sparse_feature_b200/csrc/k_sinkhorn.cu"),
@@ -122,6 +125,8 @@ def algorithmic_work(B, M, N, n_stages=18, T=100, D=256):
         "score_gemm": ("tensor", 2.0 * B * M * N * D),
         # streamed-byte model of the transport: two fp32 passes over the augmented matrix per iteration
         "sinkhorn": ("hbm", 2.0 * T * 4 * E * B),
+        # double-softmax head: the compulsory bytes (read the similarity, write log P)
+        "dsm_head": ("hbm", 8.0 * E * B),
     }
 
 
@@ -179,7 +184,7 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------------------- oracle sample
-def oracle_step(batch, weights, pair=0, stages_sampled=2, iters_sampled=10):
+def oracle_step(batch, weights, pair=0, stages_sampled=2, iters_sampled=10, head="sinkhorn"):
     """Time the float64 oracle on a bounded sample of one pair and extrapolate
     to the whole pair: encoder, `stages_sampled` attentional stages (one self,
     one cross) of the 18, projection + scores, `iters_sampled` of the 100
@@ -193,16 +198,24 @@ def oracle_step(batch, weights, pair=0, stages_sampled=2, iters_sampled=10):
     t1 = time.perf_counter()
     x0, x1 = O.attentional_gnn(x0, x1, weights, synth.H, synth.BN_EPS, n_stages=stages_sampled)
     t2 = time.perf_counter()
-    S = O.score_matrix(x0, x1, weights["Wf"], weights["bf"])
-    t3 = time.perf_counter()
-    logP = O.log_optimal_transport(S, float(weights["bin_score"]), iters_sampled)
-    t4 = time.perf_counter()
+    if head == "double_softmax":
+        logP, _, _, _ = O.double_softmax_head(x0, x1, weights["lg_Wp"], weights["lg_bp"],
+                                              weights["lg_wz"], weights["lg_bz"])
+        t3 = t4 = time.perf_counter()
+        iters_sampled = synth.SINKHORN_ITERS
+    else:
+        S = O.score_matrix(x0, x1, weights["Wf"], weights["bf"])
+        t3 = time.perf_counter()
+        logP = O.log_optimal_transport(S, float(weights["bin_score"]), iters_sampled)
+        t4 = time.perf_counter()
     O.extract_matches(logP, synth.MATCH_THRESHOLD)
     t5 = time.perf_counter()
     per_pair = ((t1 - t0) + (t2 - t1) * (synth.N_STAGES / stages_sampled) + (t3 - t2)
                 + (t4 - t3) * (synth.SINKHORN_ITERS / iters_sampled) + (t5 - t4))
+    tail = ("double-softmax head" if head == "double_softmax"
+            else f"scores, {iters_sampled} of {synth.SINKHORN_ITERS} Sinkhorn iterations")
     desc = (f"1 pair of {len(k0)}x{len(k1)}: encoder, {stages_sampled} of {synth.N_STAGES} stages, "
-            f"scores, {iters_sampled} of {synth.SINKHORN_ITERS} Sinkhorn iterations, extraction; "
+            f"{tail}, extraction; "
             f"scaled to the whole pair ({t5 - t0:.1f} s measured)")
     return per_pair, desc
 
@@ -241,10 +254,15 @@ def run_reference(args, w):
     }
 
 
-def _config(w, n_gpus):
-    return {"workload": w.name, "B_per_gpu": w.B, "M": w.M, "N": w.N, "stages": synth.N_STAGES,
-            "sinkhorn_iters": synth.SINKHORN_ITERS, "precision": w.precision,
-            "parallelism": f"replicas{n_gpus}", "l2": "flushed (256 MiB write) before every timed step"}
+def _config(w, n_gpus, head="sinkhorn"):
+    c = {"workload": w.name, "B_per_gpu": w.B, "M": w.M, "N": w.N, "stages": synth.N_STAGES,
+         "sinkhorn_iters": synth.SINKHORN_ITERS, "precision": w.precision,
+         "parallelism": f"replicas{n_gpus}", "l2": "flushed (256 MiB write) before every timed step"}
+    if head != "sinkhorn":
+        c["head"] = head
+        c["match_threshold"] = DSM_THRESHOLD
+        del c["sinkhorn_iters"]
+    return c
 
 
 def run_native(args, w):
@@ -270,10 +288,12 @@ def run_native(args, w):
     weights = synth.make_weights(0)
     batch = synth.make_batch(w, shard_pairs(B, rank), B)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        t, desc = oracle_step(batch, weights)
+        t, desc = oracle_step(batch, weights, head=args.head)
         cpu_baseline = {"value": 1.0 / t, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle", "sample": desc}
 
-    m = Matcher(weights, B, M, N, precision=w.precision)
+    dsm = args.head == "double_softmax"
+    m = Matcher(weights, B, M, N, precision=w.precision, head=args.head,
+                match_threshold=DSM_THRESHOLD if dsm else synth.MATCH_THRESHOLD)
     t = {k: torch.from_numpy(np.ascontiguousarray(batch[k])).to(dev)
          for k in ("kpts0", "conf0", "desc0", "kpts1", "conf1", "desc1")}
     logP = torch.empty((B, M + 1, N + 1), dtype=torch.float32, device=dev)
@@ -335,6 +355,8 @@ def run_native(args, w):
         step()
     torch.cuda.synchronize()
     _, per_class = timed(step, args.steps, profile=True)
+    if dsm and "sinkhorn" in per_class:
+        per_class["dsm_head"] = per_class.pop("sinkhorn")   # the assignment-step class
     m.profile(False)
     st = m.status()
     if st != 0:
@@ -414,7 +436,7 @@ def run_native(args, w):
         "vs_baseline": (value / PAGES_PAIRS_PER_S[w.name]) if w.name in PAGES_PAIRS_PER_S else None,
         "dtype": "bf16" if w.precision == "bf16" else "f32",
         "data": "synthetic (seeded keypoint pairs, random-init weights)",
-        "config": _config(w, world),
+        "config": _config(w, world, args.head),
         "roofline": roofline,
         "gnn_tensor_frac": (gnn_flops / gnn_s / 1e12 / peaks["bf16_tflops"]) if gnn_s > 0 else None,
         "kernels": breakdown,
@@ -437,6 +459,9 @@ def main():
     ap.add_argument("--workload", default="pair2048", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--head", default="sinkhorn", choices=["sinkhorn", "double_softmax"],
+                    help="matching head: dustbin + Sinkhorn (the default, the headline metric) or "
+                         "the double-softmax head")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

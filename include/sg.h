@@ -73,6 +73,13 @@ typedef enum {
                                  fp32 softmax, fp32 residual stream */
 } sg_precision_t;
 
+/* Matching head after the attentional GNN. */
+typedef enum {
+    SG_HEAD_SINKHORN = 0,        /* score matrix + dustbin + log-domain Sinkhorn (SuperGlue) */
+    SG_HEAD_DOUBLE_SOFTMAX = 1   /* double softmax + matchability (the LightGlue review's
+                                    section 2.4): no dustbin score, no iterations */
+} sg_head_t;
+
 /*
  * Weights, all HOST float32 arrays, read once by sg_create (which copies,
  * folds and packs them; the caller may free them afterwards).  Every linear
@@ -91,6 +98,11 @@ typedef enum {
  *           BatchNorm; W2 (D x 2D): second layer, bias fixed at 0.
  *   Wf, bf: final projection D x D.
  *   bin_score: the dustbin score z (alpha).
+ *   lg_Wp, lg_bp, lg_wz, lg_bz: the double-softmax head (only read when
+ *       cfg.head == SG_HEAD_DOUBLE_SOFTMAX): final projection D x D and bias
+ *       (the similarity is <m0, m1> with m = (lg_Wp x + lg_bp) / D^(1/4)),
+ *       matchability weights (D) and bias of z = lg_wz . x + lg_bz on the GNN
+ *       states.  Wf, bf and bin_score are then not used.
  */
 typedef struct {
     const float* enc_W[SG_ENC_LAYERS];
@@ -111,6 +123,10 @@ typedef struct {
     const float* Wf;
     const float* bf;
     float bin_score;
+    const float* lg_Wp;
+    const float* lg_bp;
+    const float* lg_wz;
+    float lg_bz;
 } sg_weights;
 
 /*
@@ -130,6 +146,7 @@ typedef struct {
     float img_w, img_h;      /* image size used by the keypoint normalisation */
     int norm_mode;
     int max_B, max_M, max_N;
+    int head;                /* sg_head_t; the pages' LightGlue default threshold is 0.1 */
 } sg_config;
 
 /* Create a handle on the current device: validates cfg, copies and packs the
@@ -195,6 +212,26 @@ sg_status_t sg_optimal_transport(sg_handle* h, int B, int M, int N,
  * reported an error.
  */
 sg_status_t sg_status(sg_handle* h, void* stream);
+
+/*
+ * Step 5 of the double-softmax head on given inputs (the counterpart of
+ * sg_optimal_transport for cfg.head == SG_HEAD_DOUBLE_SOFTMAX; the handle may
+ * have either head): from the similarity sim (B x M x N, float32, row-major,
+ * device) and the matchability logits z0 (B x M) and z1 (B x N), writes the
+ * (M+1) x (N+1) log assignment per pair into out_logP (NULL to skip):
+ *   real block  log_softmax over j + log_softmax over i + log sigmoid(z0_i)
+ *               + log sigmoid(z1_j);  last column log sigmoid(-z0_i);
+ *   last row    log sigmoid(-z1_j);   corner 0
+ * ("论文解读:LightGlue,让稀疏特征匹配随难度自适应地快", section 2.4), and the mutual
+ * argmax matches with the strict threshold cfg.match_threshold, as sg_match
+ * does.  Uses the handle's scratch; asynchronous on `stream`.  Errors as
+ * sg_optimal_transport (SG_ERR_SHAPE for B, M or N outside the handle's
+ * maxima or M == 0 or N == 0 with B > 0).
+ */
+sg_status_t sg_assign_double_softmax(sg_handle* h, int B, int M, int N, const float* sim,
+                                     const float* z0, const float* z1, float* out_logP,
+                                     int32_t* matches0, int32_t* matches1,
+                                     float* mscores0, float* mscores1, void* stream);
 
 /*
  * Self-test of the device-side failure detection: launches one CTA of a

@@ -26,7 +26,7 @@ STATUS = {0: "SG_OK", 1: "SG_ERR_INVALID_ARG", 2: "SG_ERR_SHAPE", 3: "SG_ERR_OOM
 EXPORTED = ["sg_create", "sg_destroy", "sg_match", "sg_match_host", "sg_scores",
             "sg_optimal_transport", "sg_status", "sg_strerror", "sg_launches_per_match",
             "sg_selftest_barrier_timeout", "sg_profile", "sg_profile_read",
-            "sg_optimal_transport_static", "sg_selftest_exp2_poly"]
+            "sg_optimal_transport_static", "sg_selftest_exp2_poly", "sg_assign_double_softmax"]
 
 KERNEL_CLASSES = ["encoder", "qkv_gemm", "attention", "mlp1_gemm", "mlp2_gemm", "proj_gemm",
                   "score_gemm", "sinkhorn"]
@@ -48,6 +48,7 @@ class SgWeights(C.Structure):
         ("W2", _FP * SG_MAX_STAGES),
         ("Wf", _FP), ("bf", _FP),
         ("bin_score", C.c_float),
+        ("lg_Wp", _FP), ("lg_bp", _FP), ("lg_wz", _FP), ("lg_bz", C.c_float),
     ]
 
 
@@ -57,7 +58,11 @@ class SgConfig(C.Structure):
         ("match_threshold", C.c_float), ("bn_eps", C.c_float), ("precision", C.c_int),
         ("img_w", C.c_float), ("img_h", C.c_float), ("norm_mode", C.c_int),
         ("max_B", C.c_int), ("max_M", C.c_int), ("max_N", C.c_int),
+        ("head", C.c_int),
     ]
+
+
+HEADS = {"sinkhorn": 0, "double_softmax": 1}
 
 
 class SgError(RuntimeError):
@@ -91,6 +96,8 @@ def load():
     lib.sg_scores.restype = i32
     lib.sg_optimal_transport.argtypes = [vp, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp]
     lib.sg_optimal_transport.restype = i32
+    lib.sg_assign_double_softmax.argtypes = [vp, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+    lib.sg_assign_double_softmax.restype = i32
     lib.sg_status.argtypes = [vp, vp]
     lib.sg_status.restype = i32
     lib.sg_strerror.argtypes = [i32]
@@ -137,7 +144,8 @@ class Matcher:
 
     def __init__(self, weights: dict, max_B: int, max_M: int, max_N: int, precision: str = "bf16",
                  n_stages: int | None = None, sinkhorn_iters: int = 100, match_threshold: float = 0.2,
-                 bn_eps: float = 1e-5, img_w: float = 640.0, img_h: float = 480.0, norm_mode: int = 0):
+                 bn_eps: float = 1e-5, img_w: float = 640.0, img_h: float = 480.0, norm_mode: int = 0,
+                 head: str = "sinkhorn"):
         lib = load()
         self._keep = []
         w = SgWeights()
@@ -164,8 +172,14 @@ class Matcher:
         w.Wf = fp(weights["Wf"])
         w.bf = fp(weights["bf"])
         w.bin_score = float(weights["bin_score"])
+        if head == "double_softmax":
+            w.lg_Wp = fp(weights["lg_Wp"])
+            w.lg_bp = fp(weights["lg_bp"])
+            w.lg_wz = fp(weights["lg_wz"])
+            w.lg_bz = float(weights["lg_bz"])
         cfg = SgConfig(256, 4, n, sinkhorn_iters, match_threshold, bn_eps,
-                       1 if precision == "bf16" else 0, img_w, img_h, norm_mode, max_B, max_M, max_N)
+                       1 if precision == "bf16" else 0, img_w, img_h, norm_mode, max_B, max_M, max_N,
+                       HEADS[head])
         h = C.c_void_p()
         _check(lib.sg_create(C.byref(w), C.byref(cfg), C.byref(h)), "sg_create")
         self._keep = []
@@ -213,6 +227,14 @@ class Matcher:
                                              _ptr(matches0), _ptr(matches1), _ptr(mscores0),
                                              _ptr(mscores1), _stream_ptr(stream)),
                "sg_optimal_transport")
+
+    def assign_double_softmax(self, sim, z0, z1, out_logP, matches0, matches1, mscores0, mscores1, stream=None):
+        """sg_assign_double_softmax on device tensors: sim (B, M, N), z0 (B, M), z1 (B, N)."""
+        B, M, N = sim.shape
+        _check(self.lib.sg_assign_double_softmax(self.h, B, M, N, _ptr(sim), _ptr(z0), _ptr(z1), _ptr(out_logP),
+                                                 _ptr(matches0), _ptr(matches1), _ptr(mscores0),
+                                                 _ptr(mscores1), _stream_ptr(stream)),
+               "sg_assign_double_softmax")
 
     def status(self, stream=None):
         return self.lib.sg_status(self.h, _stream_ptr(stream))

@@ -64,6 +64,9 @@ struct sg_handle {
   void* Wf;
   float* bf;
   float alpha;
+  float score_scale;   // 1/sqrt(D) for the Sinkhorn head; 1 when folded into Wf (double softmax)
+  float* lg_wz;        // double-softmax head: matchability weights (fp32) and bias
+  float lg_bz;
   // workspace
   float* x32;
   __nv_bfloat16* x16;
@@ -74,6 +77,9 @@ struct sg_handle {
   float* Z;
   unsigned char* sk_scratch;
   size_t sk_scratch_bytes;
+  unsigned char* dsm_scratch;   // double-softmax head
+  float* z0;                    // matchability logits (B x M), (B x N)
+  float* z1;
   unsigned* status;
   // host-buffer staging
   float *s_k0, *s_c0, *s_d0, *s_k1, *s_c1, *s_d1, *s_logP, *s_ms0, *s_ms1;
@@ -229,11 +235,28 @@ sg_status_t pack_weights(sg_handle* h, const sg_weights* w) {
     st.b1 = upload_f32(h, L1.b, &ok);
     st.W2 = upload_w(h, W2, &ok);
   }
-  if (!w->Wf || !w->bf) return SG_ERR_INVALID_ARG;
-  std::vector<double> Wf(w->Wf, w->Wf + (size_t)D * D), bf(w->bf, w->bf + D);
-  h->Wf = upload_w(h, Wf, &ok);
-  h->bf = upload_f32(h, bf, &ok);
-  h->alpha = w->bin_score;
+  if (c.head == SG_HEAD_DOUBLE_SOFTMAX) {
+    // m = (Wp x + bp) / D^(1/4) on both sides: the 1/D^(1/4) goes into the
+    // projection and the score GEMM runs unscaled
+    if (!w->lg_Wp || !w->lg_bp || !w->lg_wz) return SG_ERR_INVALID_ARG;
+    const double sc = 1.0 / std::pow((double)D, 0.25);
+    std::vector<double> Wp((size_t)D * D), bp(D), wz(D);
+    for (size_t i = 0; i < (size_t)D * D; ++i) Wp[i] = w->lg_Wp[i] * sc;
+    for (int i = 0; i < D; ++i) { bp[i] = w->lg_bp[i] * sc; wz[i] = w->lg_wz[i]; }
+    h->Wf = upload_w(h, Wp, &ok);
+    h->bf = upload_f32(h, bp, &ok);
+    h->lg_wz = upload_f32(h, wz, &ok);
+    h->lg_bz = w->lg_bz;
+    h->score_scale = 1.f;
+    h->alpha = 0.f;
+  } else {
+    if (!w->Wf || !w->bf) return SG_ERR_INVALID_ARG;
+    std::vector<double> Wf(w->Wf, w->Wf + (size_t)D * D), bf(w->bf, w->bf + D);
+    h->Wf = upload_w(h, Wf, &ok);
+    h->bf = upload_f32(h, bf, &ok);
+    h->alpha = w->bin_score;
+    h->score_scale = (float)(1.0 / std::sqrt((double)D));
+  }
   return ok ? SG_OK : SG_ERR_OOM;
 }
 
@@ -339,7 +362,7 @@ cudaError_t run_network(sg_handle* h, int B, int M, int N, const Inputs& in, flo
   g.out = S; g.ldo = lds;
   g.rows = M; g.cols = N; g.K = kD;
   g.strideA = (long long)P * kD; g.strideW = (long long)P * kD; g.strideO = strideS;
-  g.scale = (float)(1.0 / std::sqrt((double)kD));
+  g.scale = h->score_scale;
   return gemm(h, g, EPI_SCALE, false, B, s, launches, K_SCORE);
 }
 
@@ -467,7 +490,8 @@ const char* sg_strerror(sg_status_t s) {
 
 int sg_launches_per_match(const sg_handle* h, int B, int M, int N) {
   if (!h || B == 0 || M == 0 || N == 0) return 0;
-  return (h->use_tc ? 6 : 4) + 4 * h->cfg.n_stages;
+  const int net = (h->use_tc ? 5 : 3) + 4 * h->cfg.n_stages;   // encoder .. score GEMM
+  return net + (h->cfg.head == SG_HEAD_DOUBLE_SOFTMAX ? 7 : 1);  // matchability + 6 head kernels, or Sinkhorn
 }
 
 sg_status_t sg_create(const sg_weights* w, const sg_config* cfg, sg_handle** out) {
@@ -478,7 +502,8 @@ sg_status_t sg_create(const sg_weights* w, const sg_config* cfg, sg_handle** out
   if (cfg->n_stages < 1 || cfg->n_stages > SG_MAX_STAGES || cfg->sinkhorn_iters < 0 ||
       cfg->max_B < 0 || cfg->max_M < 0 || cfg->max_N < 0 || !(cfg->bn_eps >= 0.f) ||
       !(cfg->img_w > 0.f) || !(cfg->img_h > 0.f) || (cfg->norm_mode != 0 && cfg->norm_mode != 1) ||
-      (cfg->precision != SG_PRECISION_FP32 && cfg->precision != SG_PRECISION_BF16))
+      (cfg->precision != SG_PRECISION_FP32 && cfg->precision != SG_PRECISION_BF16) ||
+      (cfg->head != SG_HEAD_SINKHORN && cfg->head != SG_HEAD_DOUBLE_SOFTMAX))
     return SG_ERR_INVALID_ARG;
   if (cfg->max_N > sinkhorn_max_columns()) return SG_ERR_UNSUPPORTED;   // transport kernel columns
   int dev = 0;
@@ -529,6 +554,9 @@ sg_status_t sg_create(const sg_weights* w, const sg_config* cfg, sg_handle** out
   h->Z = (float*)al(Bm * Mm * ((Nm + 3) & ~(size_t)3) * 4);
   h->sk_scratch_bytes = sinkhorn_scratch_bytes((int)Bm, (int)Mm, (int)Nm);
   h->sk_scratch = (unsigned char*)al(h->sk_scratch_bytes);
+  h->dsm_scratch = (unsigned char*)al(dsm_scratch_bytes((int)Bm, (int)Mm, (int)Nm));
+  h->z0 = (float*)al(Bm * Mm * 4);
+  h->z1 = (float*)al(Bm * Nm * 4);
   h->status = (unsigned*)al(sizeof(unsigned));
   h->s_k0 = (float*)al(Bm * Mm * 2 * 4);
   h->s_c0 = (float*)al(Bm * Mm * 4);
@@ -600,6 +628,20 @@ sg_status_t sg_optimal_transport(sg_handle* h, int B, int M, int N, const float*
                                    matches1, mscores0, mscores1, (cudaStream_t)stream, &launches));
 }
 
+sg_status_t sg_assign_double_softmax(sg_handle* h, int B, int M, int N, const float* sim, const float* z0,
+                                     const float* z1, float* out_logP, int32_t* matches0, int32_t* matches1,
+                                     float* mscores0, float* mscores1, void* stream) {
+  sg_status_t st = check_shape(h, B, M, N);
+  if (st != SG_OK) return st;
+  if (B == 0) return SG_OK;
+  if (M == 0 || N == 0) return SG_ERR_SHAPE;
+  if (!sim || !z0 || !z1 || !matches0 || !matches1 || !mscores0 || !mscores1) return SG_ERR_INVALID_ARG;
+  int launches = 0;
+  return cuda_err(h, launch_dsm_assign(sim, N, (long long)M * N, B, M, N, z0, z1, h->cfg.match_threshold,
+                                       out_logP, matches0, matches1, mscores0, mscores1, h->dsm_scratch,
+                                       (cudaStream_t)stream, &launches));
+}
+
 sg_status_t sg_match(sg_handle* h, int B, int M, int N, const float* kpts0, const float* conf0,
                      const float* desc0, const float* kpts1, const float* conf1, const float* desc1,
                      float* out_logP, int32_t* matches0, int32_t* matches1, float* mscores0,
@@ -624,6 +666,17 @@ sg_status_t sg_match(sg_handle* h, int B, int M, int N, const float* kpts0, cons
     h->prof_n = 0;
     cudaError_t e = run_network(h, B, M, N, in, h->Z, lds, strideS, cs, launches);
     if (e != cudaSuccess) return e;
+    if (h->cfg.head == SG_HEAD_DOUBLE_SOFTMAX) {
+      // matchability from the final GNN states, then the closed-form assignment
+      mark(h, cs, K_SINKHORN);
+      e = launch_dsm_matchability(h->x32, B, M, N, h->lg_wz, h->lg_bz, h->z0, h->z1, cs);
+      ++*launches;
+      if (e != cudaSuccess) return e;
+      e = launch_dsm_assign(h->Z, lds, strideS, B, M, N, h->z0, h->z1, h->cfg.match_threshold, out_logP,
+                            matches0, matches1, mscores0, mscores1, h->dsm_scratch, cs, launches);
+      mark(h, cs, K_END);
+      return e;
+    }
     return run_transport(h, B, M, N, h->Z, lds, strideS, out_logP, matches0, matches1, mscores0,
                          mscores1, cs, launches);
   });

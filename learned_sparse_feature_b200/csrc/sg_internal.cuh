@@ -113,6 +113,14 @@ cudaError_t sinkhorn_prepare(int num_sms);   // kernel attributes (called once, 
 int sinkhorn_max_columns();                  // largest N the transport kernel supports
 size_t sinkhorn_scratch_bytes(int B, int M, int N);
 size_t sinkhorn_acc_floats_per_buffer(int N);   // column accumulator floats per (pair, rotation)
+// Double-softmax matching head (k_dsm.cu).
+size_t dsm_scratch_bytes(int B, int M, int N);
+cudaError_t launch_dsm_matchability(const float* x32, int B, int M, int N, const float* wz, float bz, float* z0,
+                                    float* z1, cudaStream_t s);
+cudaError_t launch_dsm_assign(const float* S, long long lds, long long strideS, int B, int M, int N,
+                              const float* z0, const float* z1, float threshold, float* logP, int32_t* matches0,
+                              int32_t* matches1, float* mscores0, float* mscores1, void* scratch, cudaStream_t s,
+                              int* launches);
 cudaError_t launch_exp2_poly_selftest(const float* x, float* y, int n, cudaStream_t s);
 cudaError_t launch_barrier_selftest(unsigned* scratch, unsigned* status, unsigned long long timeout_ns,
                                     int* returned, cudaStream_t s);
