@@ -35,7 +35,8 @@ namespace {
 
 constexpr int BM = 128;
 constexpr int BK = 64;                   // one 128-byte swizzle atom of bf16
-constexpr int kThreads = 192;                // producer, MMA, 4 epilogue warps
+constexpr int kEpiWarps = 8;                 // two per TMEM lane quarter
+constexpr int kThreads = 64 + 32 * kEpiWarps;    // producer, MMA, epilogue warps
 constexpr unsigned kErrGemmWait = 4u;    // status bit: a GEMM pipeline wait ran out
 
 struct TcArgs {
@@ -50,12 +51,14 @@ struct TcArgs {
   long long strideO;
   float scale;
   unsigned* status;
+  int b_const;           // W is constant (weights), not an output of an earlier kernel
 };
 
-// Epilogue staging of one epilogue warp: two buffer sets, each a 32-row chunk of
-// the output (fp32 rows of 128 B or bf16 rows of 64 B) and, for the residual
-// epilogue, its bf16 copy and the fp32 residual input.  Offsets are multiples
-// of 1024 B (the swizzle atoms of the TMA boxes).
+// Epilogue staging of one epilogue warp: one buffer set, a 32-row chunk of the
+// output (fp32 rows of 128 B or bf16 rows of 64 B) and, for the residual
+// epilogue, its bf16 copy and the fp32 residual input.  The two warps of a lane
+// quarter alternate chunks, so a quarter's chunks are double-buffered.  Offsets
+// are multiples of 1024 B (the swizzle atoms of the TMA boxes).
 template <int EPI>
 struct EpiStage {
   static constexpr bool F32 = EPI == EPI_SCALE || EPI == EPI_RESIDUAL;
@@ -65,8 +68,7 @@ struct EpiStage {
   static constexpr int OUT2_OFF = OUT;
   static constexpr int RES_OFF = OUT + OUT2;
   static constexpr int BUF = OUT + OUT2 + RES;
-  static constexpr int WARP = 2 * BUF;
-  static constexpr int BYTES = 4 * WARP;
+  static constexpr int BYTES = kEpiWarps * BUF;
 };
 
 constexpr int kMaxDynSmem = 224 * 1024;
@@ -95,7 +97,7 @@ __device__ __forceinline__ bool epi_all(bool v) {
   asm volatile(
       "{\n\t.reg .pred p, q;\n\t"
       "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.and.pred q, 1, 128, p;\n\t"
+      "bar.red.and.pred q, 1, 256, p;\n\t"
       "selp.u32 %0, 1, 0, q;\n\t}"
       : "=r"(r)
       : "r"((uint32_t)v)
@@ -125,7 +127,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
   __shared__ __align__(8) uint64_t empty_bar[STAGES];
   __shared__ __align__(8) uint64_t tfull_bar[2];
   __shared__ __align__(8) uint64_t tempty_bar[2];
-  __shared__ __align__(8) uint64_t res_bar[4][2];   // residual chunk loads, per epilogue warp and buffer
+  __shared__ __align__(8) uint64_t res_bar[kEpiWarps];   // residual chunk loads, per epilogue warp
   __shared__ __align__(16) float s_bias[2][BN];   // bias of the tile, by accumulator buffer
   __shared__ uint32_t tmem_slot;
   __shared__ int s_abort;
@@ -148,12 +150,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
     }
     for (int b = 0; b < 2; ++b) {
       tc::mbar_init(&tfull_bar[b], 1);
-      tc::mbar_init(&tempty_bar[b], 4);          // one arrival per epilogue warp
+      tc::mbar_init(&tempty_bar[b], kEpiWarps);  // one arrival per epilogue warp
     }
-    for (int w = 0; w < 4; ++w) {
-      tc::mbar_init(&res_bar[w][0], 1);
-      tc::mbar_init(&res_bar[w][1], 1);
-    }
+    for (int w = 0; w < kEpiWarps; ++w) tc::mbar_init(&res_bar[w], 1);
     tc::fence_barrier_init();
     s_abort = 0;
   }
@@ -169,11 +168,26 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = tmem_slot;
-  pdl_wait();                                    // the previous kernel's outputs are complete
+  // the previous kernel's outputs must be complete before they are read and
+  // before this kernel's outputs overwrite anything it still reads; the
+  // producer first fetches constant weight tiles, which need neither
+  if (!(warp == 0 && lane == 0)) pdl_wait();
 
   if (warp == 0) {
     if (lane == 0) {
       // ---------------- TMA producer
+      int pre = 0;                               // ring stages whose W tile is already in flight
+      if (g.b_const && (int)blockIdx.x < ntiles) {
+        const int t = blockIdx.x;
+        const int tn = t % ntn, bz = t / (ntn * ntm);
+        const int b_row = g.b_row0 + bz * g.b_batch_rows + tn * BN;
+        pre = nkb < STAGES ? nkb : STAGES;
+        for (int kb = 0; kb < pre; ++kb) {
+          tc::mbar_arrive_expect_tx(&full_bar[kb], SM::STAGE_BYTES);
+          tc::tma_load_2d(&tmB, &full_bar[kb], sbase + kb * SM::STAGE_BYTES + SM::A_BYTES, kb * BK, b_row);
+        }
+      }
+      pdl_wait();
       int it = 0;
       for (int t = blockIdx.x; t < ntiles && !s_abort; t += gridDim.x) {
         const int tn = t % ntn, tm = (t / ntn) % ntm, bz = t / (ntn * ntm);
@@ -188,10 +202,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
           }
           uint8_t* sa = sbase + s * SM::STAGE_BYTES;
           uint8_t* sb = sa + SM::A_BYTES;
-          tc::mbar_arrive_expect_tx(&full_bar[s], SM::STAGE_BYTES);
+          if (it >= pre) tc::mbar_arrive_expect_tx(&full_bar[s], SM::STAGE_BYTES);
           if (kb < nkb0) tc::tma_load_2d(&tmA0, &full_bar[s], sa, kb * BK, a_row);
           else tc::tma_load_2d(&tmA1, &full_bar[s], sa, (kb - nkb0) * BK, a_row);
-          tc::tma_load_2d(&tmB, &full_bar[s], sb, kb * BK, b_row);
+          if (it >= pre) tc::tma_load_2d(&tmB, &full_bar[s], sb, kb * BK, b_row);
         }
       }
       // drain: copies in flight must land before the CTA may exit
@@ -237,17 +251,20 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
       }
     }
   } else {
-    // ---------------- epilogue warps 2..5: TMEM lane quarter = warp % 4
+    // ---------------- epilogue warps 2..9: TMEM lane quarter q = warp % 4;
+    // the two warps of a quarter (hf = 0, 1) take alternate 32-column chunks.
     // While the MMA warp accumulates a tile, these warps stage its bias in
-    // shared memory and (residual) start the TMA loads of the first two
-    // residual chunks.  Warp q owns tile rows 32q .. 32q+31, thread = row.
+    // shared memory and (residual) start the TMA load of their first residual
+    // chunk.  Thread = tile row 32q + lane.
     const int q = warp & 3;
-    const int et = threadIdx.x - 64;             // 0..127
-    uint8_t* wbuf = sbase + SM::EPI_OFF + q * ES::WARP;
-    constexpr int NCH = BN / 32;                 // 32-column chunks per tile
-    int chunk = 0;                               // chunks done by this warp (buffer = chunk & 1)
-    uint32_t res_par = 0;                        // residual barrier parities, bit per buffer
-    uint32_t res_pend = 0;                       // residual loads issued and not yet waited for
+    const int ew = warp - 2;                     // 0..7: staging slot
+    const int hf = ew >> 2;                      // which chunks of the quarter
+    const int et = threadIdx.x - 64;             // 0..255
+    uint8_t* sbuf = sbase + SM::EPI_OFF + ew * ES::BUF;
+    constexpr int NCH = BN / 32;                 // 32-column chunks per tile (even)
+    constexpr int MYCH = NCH / 2;                // chunks of one warp per tile
+    uint32_t res_par = 0;                        // residual barrier parity
+    bool res_pend = false;                       // a residual load issued and not yet waited for
     int i = 0;
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++i) {
       const int b = i & 1;
@@ -255,85 +272,83 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
       const int n0 = tn * BN;
       const int row0 = tm * BM + q * 32;         // first row of this warp's chunks
       if (EPI == EPI_BIAS || EPI == EPI_BIAS_RELU) {
-        for (int c = et; c < BN; c += 128) s_bias[b][c] = (n0 + c < g.cols) ? __ldg(g.bias + n0 + c) : 0.f;
+        for (int c = et; c < BN; c += 32 * kEpiWarps)
+          s_bias[b][c] = (n0 + c < g.cols) ? __ldg(g.bias + n0 + c) : 0.f;
       }
       if (EPI == EPI_RESIDUAL && lane == 0) {
-        for (int c = 0; c < 2 && c < NCH; ++c) {
-          const int bb = (chunk + c) & 1;
-          tc::mbar_arrive_expect_tx(&res_bar[q][bb], 4096);
-          tc::tma_load_3d(&tmO, &res_bar[q][bb], wbuf + bb * ES::BUF + ES::RES_OFF, n0 + 32 * c, row0, bz);
-          res_pend |= 1u << bb;
-        }
+        tc::mbar_arrive_expect_tx(&res_bar[ew], 4096);
+        tc::tma_load_3d(&tmO, &res_bar[ew], sbuf + ES::RES_OFF, n0 + 32 * hf, row0, bz);
+        res_pend = true;
       }
       const bool got = tc::mbar_wait(&tfull_bar[b], (i >> 1) & 1, g.status, kErrGemmWait);
-      // one barrier of the 128 epilogue threads per tile: publishes the staged
-      // bias and makes the go / stop decision the same for all of them
+      // one barrier of the epilogue threads per tile: publishes the staged bias
+      // and makes the go / stop decision the same for all of them
       if (!epi_all(got && !s_abort)) break;
       tc::tc_fence_after();
       const uint32_t trow = tmem + b * BNA + ((uint32_t)(q * 32) << 16);
       bool ok = true;
-      // chunk ci's accumulator columns arrive while chunk ci - 1 is processed
+      // the next chunk's accumulator columns arrive while a chunk is processed
       float va[32], vb[32];
-      tc::tmem_ld32_async(trow, va);            // warp-collective: every lane takes part
+      tc::tmem_ld32_async(trow + hf * 32, va);  // warp-collective: every lane takes part
 #pragma unroll
-      for (int ci = 0; ci < NCH; ++ci, ++chunk) {
-        const int bb = chunk & 1;
-        uint8_t* sbuf = wbuf + bb * ES::BUF;
-        float (&v)[32] = (ci & 1) ? vb : va;
+      for (int k = 0; k < MYCH; ++k) {
+        const int ci = hf + 2 * k;
+        float (&v)[32] = (k & 1) ? vb : va;
         tc::tmem_wait_ld(v);
-        if (ci + 1 < NCH) tc::tmem_ld32_async(trow + (ci + 1) * 32, (ci & 1) ? va : vb);
-        // the store issued from this buffer two chunks ago must have read it
-        if (lane == 0) tc::bulk_wait_read<1>();
+        if (k + 1 < MYCH) tc::tmem_ld32_async(trow + (ci + 2) * 32, (k & 1) ? va : vb);
+        // the store issued from this buffer (this warp's previous chunk) must have read it
+        if (lane == 0) tc::bulk_wait_read<0>();
         __syncwarp();
         if (EPI == EPI_BIAS || EPI == EPI_BIAS_RELU) {
           // bf16 row of 64 B, 64-byte swizzle: 16-byte chunk k at k ^ ((row >> 1) & 3)
           const float4* b4 = reinterpret_cast<const float4*>(s_bias[b] + ci * 32);
           uint8_t* rowp = sbuf + lane * 64;
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
+          for (int kk = 0; kk < 4; ++kk) {
             uint32_t pk[4];
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-              const float4 bb4 = b4[2 * k + h];
-              float x0 = v[8 * k + 4 * h] + bb4.x, x1 = v[8 * k + 4 * h + 1] + bb4.y;
-              float x2 = v[8 * k + 4 * h + 2] + bb4.z, x3 = v[8 * k + 4 * h + 3] + bb4.w;
+              const float4 bb4 = b4[2 * kk + h];
+              float x0 = v[8 * kk + 4 * h] + bb4.x, x1 = v[8 * kk + 4 * h + 1] + bb4.y;
+              float x2 = v[8 * kk + 4 * h + 2] + bb4.z, x3 = v[8 * kk + 4 * h + 3] + bb4.w;
               if (EPI == EPI_BIAS_RELU) {
                 x0 = fmaxf(x0, 0.f); x1 = fmaxf(x1, 0.f); x2 = fmaxf(x2, 0.f); x3 = fmaxf(x3, 0.f);
               }
               pk[2 * h] = tc::pack_bf16x2(x0, x1);
               pk[2 * h + 1] = tc::pack_bf16x2(x2, x3);
             }
-            *reinterpret_cast<uint4*>(rowp + ((k ^ ((lane >> 1) & 3)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            *reinterpret_cast<uint4*>(rowp + ((kk ^ ((lane >> 1) & 3)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
           }
         } else if (EPI == EPI_SCALE) {
           // fp32 row of 128 B, 128-byte swizzle: 16-byte chunk k at k ^ (row & 7)
           uint8_t* rowp = sbuf + lane * 128;
 #pragma unroll
-          for (int k = 0; k < 8; ++k)
-            *reinterpret_cast<float4*>(rowp + ((k ^ (lane & 7)) << 4)) =
-                make_float4(v[4 * k] * g.scale, v[4 * k + 1] * g.scale, v[4 * k + 2] * g.scale, v[4 * k + 3] * g.scale);
+          for (int kk = 0; kk < 8; ++kk)
+            *reinterpret_cast<float4*>(rowp + ((kk ^ (lane & 7)) << 4)) =
+                make_float4(v[4 * kk] * g.scale, v[4 * kk + 1] * g.scale, v[4 * kk + 2] * g.scale,
+                            v[4 * kk + 3] * g.scale);
         } else {
           // residual: x (fp32) += acc, and its bf16 copy
-          ok = tc::mbar_wait(&res_bar[q][bb], (res_par >> bb) & 1u, g.status, kErrGemmWait);
-          res_par ^= 1u << bb;
-          res_pend &= ~(1u << bb);
+          ok = tc::mbar_wait(&res_bar[ew], res_par, g.status, kErrGemmWait);
+          res_par ^= 1u;
+          res_pend = false;
           const uint8_t* rin = sbuf + ES::RES_OFF + lane * 128;
           uint8_t* rout = sbuf + lane * 128;
           uint8_t* rout2 = sbuf + ES::OUT2_OFF + lane * 64;
           uint32_t pk[16];
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const int off = (k ^ (lane & 7)) << 4;
+          for (int kk = 0; kk < 8; ++kk) {
+            const int off = (kk ^ (lane & 7)) << 4;
             float4 r = *reinterpret_cast<const float4*>(rin + off);
-            r.x += v[4 * k]; r.y += v[4 * k + 1]; r.z += v[4 * k + 2]; r.w += v[4 * k + 3];
+            r.x += v[4 * kk]; r.y += v[4 * kk + 1]; r.z += v[4 * kk + 2]; r.w += v[4 * kk + 3];
             *reinterpret_cast<float4*>(rout + off) = r;
-            pk[2 * k] = tc::pack_bf16x2(r.x, r.y);
-            pk[2 * k + 1] = tc::pack_bf16x2(r.z, r.w);
+            pk[2 * kk] = tc::pack_bf16x2(r.x, r.y);
+            pk[2 * kk + 1] = tc::pack_bf16x2(r.z, r.w);
           }
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            *reinterpret_cast<uint4*>(rout2 + ((k ^ ((lane >> 1) & 3)) << 4)) =
-                make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+          for (int kk = 0; kk < 4; ++kk)
+            *reinterpret_cast<uint4*>(rout2 + ((kk ^ ((lane >> 1) & 3)) << 4)) =
+                make_uint4(pk[4 * kk], pk[4 * kk + 1], pk[4 * kk + 2], pk[4 * kk + 3]);
         }
         tc::fence_proxy_async_smem();           // generic writes -> async-proxy reads
         __syncwarp();
@@ -344,11 +359,11 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
             if (EPI == EPI_RESIDUAL) tc::tma_store_3d(&tmO2, sbuf + ES::OUT2_OFF, n0 + ci * 32, row0, bz);
           }
           tc::bulk_commit();
-          if (EPI == EPI_RESIDUAL && ci + 2 < NCH) {
-            // this buffer's residual input is consumed: fetch the chunk after next
-            tc::mbar_arrive_expect_tx(&res_bar[q][bb], 4096);
-            tc::tma_load_3d(&tmO, &res_bar[q][bb], sbuf + ES::RES_OFF, n0 + 32 * (ci + 2), row0, bz);
-            res_pend |= 1u << bb;
+          if (EPI == EPI_RESIDUAL && k + 1 < MYCH) {
+            // this warp's residual input is consumed: fetch its next chunk
+            tc::mbar_arrive_expect_tx(&res_bar[ew], 4096);
+            tc::tma_load_3d(&tmO, &res_bar[ew], sbuf + ES::RES_OFF, n0 + 32 * (ci + 2), row0, bz);
+            res_pend = true;
           }
         }
       }
@@ -358,11 +373,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
       if (!ok) s_abort = 1;
     }
     // stores must be complete and residual loads landed before the CTA exits
-    // (a break above can leave prefetched residual chunks in flight)
+    // (a break above can leave a prefetched residual chunk in flight)
     if (lane == 0) {
       tc::bulk_wait_all();
-      for (int bb = 0; bb < 2; ++bb)
-        if ((res_pend >> bb) & 1u) tc::mbar_wait(&res_bar[q][bb], (res_par >> bb) & 1u, g.status, kErrGemmWait);
+      if (res_pend) tc::mbar_wait(&res_bar[ew], res_par, g.status, kErrGemmWait);
     }
   }
   tc::tc_fence_before();
@@ -520,6 +534,7 @@ cudaError_t launch_gemm_tc(const GemmArgs& g, int epi, int batch, cudaStream_t s
   t.b_row0 = 0;
   t.bias = g.bias; t.out = g.out; t.out2 = g.out2; t.ldo = g.ldo; t.strideO = g.strideO;
   t.scale = g.scale; t.status = status;
+  t.b_const = g.w_dynamic ? 0 : 1;
   // outputs: bf16 (bias epilogues), fp32 scores, fp32 residual stream + its bf16 copy
   CUtensorMap o, o2;
   const bool f32 = epi == EPI_SCALE || epi == EPI_RESIDUAL;

@@ -363,6 +363,7 @@ cudaError_t run_network(sg_handle* h, int B, int M, int N, const Inputs& in, flo
   g.rows = M; g.cols = N; g.K = kD;
   g.strideA = (long long)P * kD; g.strideW = (long long)P * kD; g.strideO = strideS;
   g.scale = h->score_scale;
+  g.w_dynamic = 1;   // W = f_B, the projection just computed
   return gemm(h, g, EPI_SCALE, false, B, s, launches, K_SCORE);
 }
 

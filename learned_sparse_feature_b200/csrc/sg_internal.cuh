@@ -44,6 +44,7 @@ struct GemmArgs {
   int rows, cols, K;
   long long strideA, strideW, strideO;
   float scale;
+  int w_dynamic;   // W is written by an earlier kernel of the pass (the score GEMM's f_B), not a weight
 };
 
 // Attention over the stacked state of B pairs: rows [b*P, b*P+M) are image A of
