@@ -108,6 +108,26 @@ __device__ __forceinline__ float row_max(const float (&s)[KT]) {
 // EMU of every 8 pairs take the FMA-pipe exponential, the rest the MUFU.
 template <int EMU>
 __device__ __forceinline__ float exp_row(const float (&s)[KT], float scale, float m, uint32_t tp) {
+  if (EMU == 0) {
+    // all on the MUFU: one FFMA, one ex2 and one FADD per score, four
+    // independent sums (no register-pair packing in the dependency chain)
+    const float nm = -m;
+    float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+#pragma unroll
+    for (int cc = 0; cc < KT / 16; ++cc) {
+      uint32_t pk[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int i = cc * 16 + 2 * e;
+        const float p0 = fast_ex2(fmaf(s[i], scale, nm));
+        const float p1 = fast_ex2(fmaf(s[i + 1], scale, nm));
+        if (e & 1) { s2 += p0; s3 += p1; } else { s0 += p0; s1 += p1; }
+        pk[e] = tc::pack_bf16x2(p0, p1);
+      }
+      tc::tmem_st8(tp + cc * 8, pk);
+    }
+    return (s0 + s1) + (s2 + s3);
+  }
   const uint64_t sc2 = tc::f2(scale, scale);
   const uint64_t nm2 = tc::f2(-m, -m);
   uint64_t sa = tc::f2(0.f, 0.f), sb = sa;
