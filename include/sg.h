@@ -256,14 +256,23 @@ sg_status_t sg_selftest_barrier_timeout(sg_handle* h, unsigned timeout_us, void*
 sg_status_t sg_selftest_exp2_poly(const float* x, float* y, int n, void* stream);
 
 /*
- * Per-kernel timing.  While enabled, sg_match records a CUDA event before every
+ * Per-kernel timing.  enable = 1: sg_match records a CUDA event before every
  * kernel (and the Sinkhorn scratch clear) and one after the last; the events
- * are part of the captured graph.  After the stream has been synchronised,
- * sg_profile_read sums the event intervals of the last sg_match by kernel
- * class: 0 encoder, 1 q|k|v GEMM, 2 attention, 3 update-MLP layer 1 GEMM,
- * 4 update-MLP layer 2 GEMM, 5 final projection GEMM, 6 score GEMM,
- * 7 Sinkhorn + extraction.  ms_by_class and launches_by_class need n_classes
- * >= 8 entries; returns the number of classes written, or -1.
+ * are part of the captured graph.  An event between two kernels also ends the
+ * programmatic dependent launch overlap between them, so the per-class times
+ * add up to more than the pass.  enable = 2 (segment mode): events only where
+ * the pass moves from the encoder to the GNN, from the GNN to the assignment
+ * step, and at the end, so the GNN's launches run chained as without timing.
+ * enable = 0 turns timing off; other values return SG_ERR_INVALID_ARG.
+ * After the stream has been synchronised, sg_profile_read sums the event
+ * intervals of the last sg_match by class: 0 encoder, 1 q|k|v GEMM,
+ * 2 attention, 3 update-MLP layer 1 GEMM, 4 update-MLP layer 2 GEMM, 5 final
+ * projection GEMM, 6 score GEMM, 7 Sinkhorn + extraction (or the
+ * double-softmax head), 8 the whole GNN segment, classes 1-6 back to back
+ * (segment mode only; classes 1-6 stay 0 there).  launches_by_class counts the
+ * intervals.  ms_by_class and launches_by_class need n_classes >= 8 entries
+ * (class 8 is written when n_classes >= 9); returns the number of classes
+ * written, or -1.
  */
 sg_status_t sg_profile(sg_handle* h, int enable);
 int sg_profile_read(sg_handle* h, float* ms_by_class, int* launches_by_class, int n_classes);

@@ -29,7 +29,7 @@ EXPORTED = ["sg_create", "sg_destroy", "sg_match", "sg_match_host", "sg_scores",
             "sg_optimal_transport_static", "sg_selftest_exp2_poly", "sg_assign_double_softmax"]
 
 KERNEL_CLASSES = ["encoder", "qkv_gemm", "attention", "mlp1_gemm", "mlp2_gemm", "proj_gemm",
-                  "score_gemm", "sinkhorn"]
+                  "score_gemm", "sinkhorn", "gnn"]
 
 _FP = C.POINTER(C.c_float)
 
@@ -242,8 +242,11 @@ class Matcher:
     def selftest_barrier_timeout(self, timeout_us=20000, stream=None):
         return self.lib.sg_selftest_barrier_timeout(self.h, timeout_us, _stream_ptr(stream))
 
-    def profile(self, enable: bool):
-        _check(self.lib.sg_profile(self.h, 1 if enable else 0), "sg_profile")
+    def profile(self, enable, segments: bool = False):
+        """Per-kernel timing on (events before every kernel) or off; with
+        segments=True only the encoder / GNN / assignment boundaries are timed."""
+        mode = (2 if segments else 1) if enable else 0
+        _check(self.lib.sg_profile(self.h, mode), "sg_profile")
 
     def profile_read(self):
         """{class: (ms, launches)} of the last sg_match (stream must be synchronised)."""

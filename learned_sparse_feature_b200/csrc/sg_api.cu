@@ -92,8 +92,10 @@ struct sg_handle {
   cudaGraphExec_t gexec;
   std::vector<void*> allocs;
   sg_status_t sticky;
-  // per-kernel timing (events between launches, also captured into graphs)
-  bool profiling;
+  // per-kernel timing (events between launches, also captured into graphs);
+  // profiling 1 = an event before every kernel, 2 = at segment boundaries only
+  int profiling;
+  int prof_seg;
   std::vector<cudaEvent_t> prof_ev;
   std::vector<int> prof_cls;
   int prof_n;
@@ -108,10 +110,19 @@ sg_status_t cuda_err(sg_handle* h, cudaError_t e) {
 }
 
 // Kernel classes of the per-kernel timing (sg_profile_read).
-enum KClass { K_ENCODER = 0, K_QKV, K_ATTN, K_MLP1, K_MLP2, K_PROJ, K_SCORE, K_SINKHORN, K_END };
+// K_GNN is the q|k|v-to-score segment timed as one interval (segment mode).
+enum KClass { K_ENCODER = 0, K_QKV, K_ATTN, K_MLP1, K_MLP2, K_PROJ, K_SCORE, K_SINKHORN, K_GNN, K_END };
 
 void mark(sg_handle* h, cudaStream_t s, int cls) {
   if (!h->profiling) return;
+  if (h->profiling == 2) {
+    // one event where the pass moves from the encoder to the GNN, from the GNN
+    // to the assignment step, and at the end: the GNN's launches stay chained
+    // (programmatic dependent launch) as they are without profiling
+    if (cls >= K_QKV && cls <= K_SCORE) cls = K_GNN;
+    if (h->prof_n > 0 && cls == h->prof_seg) return;
+    h->prof_seg = cls;
+  }
   if (h->prof_n >= (int)h->prof_ev.size()) return;
   cudaEventRecordWithFlags(h->prof_ev[h->prof_n], s, cudaEventRecordExternal);
   h->prof_cls[h->prof_n] = cls;
@@ -659,7 +670,7 @@ sg_status_t sg_match(sg_handle* h, int B, int M, int N, const float* kpts0, cons
   const long long strideS = (long long)M * lds;
   Inputs in{kpts0, conf0, desc0, kpts1, conf1, desc1};
   GraphKey key{};
-  key.B = B; key.M = M; key.N = N; key.kind = h->profiling ? 2 : 1;
+  key.B = B; key.M = M; key.N = N; key.kind = 1 + h->profiling;
   const void* ps[12] = {kpts0, conf0, desc0, kpts1, conf1, desc1, out_logP, matches0, matches1,
                         mscores0, mscores1, nullptr};
   std::memcpy(key.p, ps, sizeof(ps));
@@ -756,13 +767,15 @@ sg_status_t sg_profile(sg_handle* h, int enable) {
     for (int i = 0; i < n; ++i)
       if (cudaEventCreate(&h->prof_ev[i]) != cudaSuccess) return cuda_err(h, cudaGetLastError());
   }
-  h->profiling = enable != 0;
+  if (enable < 0 || enable > 2) return SG_ERR_INVALID_ARG;
+  h->profiling = enable;
   h->prof_n = 0;
   return SG_OK;
 }
 
 int sg_profile_read(sg_handle* h, float* ms_by_class, int* launches_by_class, int n_classes) {
-  if (!h || !ms_by_class || !launches_by_class || n_classes < K_END) return -1;
+  if (!h || !ms_by_class || !launches_by_class || n_classes < K_GNN) return -1;
+  if (n_classes > K_END) n_classes = K_END;
   for (int c = 0; c < n_classes; ++c) { ms_by_class[c] = 0.f; launches_by_class[c] = 0; }
   for (int i = 0; i + 1 < h->prof_n; ++i) {
     float ms = 0.f;
@@ -771,9 +784,9 @@ int sg_profile_read(sg_handle* h, float* ms_by_class, int* launches_by_class, in
       return -1;
     }
     const int c = h->prof_cls[i];
-    if (c >= 0 && c < K_END) { ms_by_class[c] += ms; launches_by_class[c] += 1; }
+    if (c >= 0 && c < n_classes) { ms_by_class[c] += ms; launches_by_class[c] += 1; }
   }
-  return K_END;
+  return n_classes;
 }
 
 sg_status_t sg_status(sg_handle* h, void* stream) {

@@ -350,3 +350,29 @@ def test_attention_max_renewal_path(dev, weights, monkeypatch):
     assert np.abs(out[0] - out[1]).max() < 2e-2 * max(1.0, np.abs(out[1]).max() / 10)
     ref = _oracle(batch, weights, 0, n_stages=2)["scores"]
     assert np.abs(out[1][0] - ref).max() < 5e-2
+
+
+# --------------------------------------------------------------------------- timing hooks
+def test_profile_modes_record_classes_and_segments(dev, weights):
+    batch = _random_batch(1, 200, 150, seed=8)
+    m = _matcher(weights, 1, 200, 150, "bf16", n_stages=4)
+    ref = _run(m, batch)
+    m.profile(True)
+    out = _run(m, batch)
+    per_kernel = m.profile_read()
+    m.profile(True, segments=True)
+    out_seg = _run(m, batch)
+    per_seg = m.profile_read()
+    m.profile(False)
+    # timing events do not change the results
+    for o in (out, out_seg):
+        np.testing.assert_array_equal(o["matches0"], ref["matches0"])
+    assert per_kernel["attention"][1] == 4 and per_kernel["qkv_gemm"][1] == 4
+    assert per_kernel["gnn"] == (0.0, 0)
+    # segment mode: encoder, the GNN as one interval, the assignment step
+    assert per_seg["gnn"][1] == 1 and per_seg["gnn"][0] > 0
+    assert per_seg["encoder"][1] == 1 and per_seg["sinkhorn"][1] == 1
+    for k in ("qkv_gemm", "attention", "mlp1_gemm", "mlp2_gemm", "proj_gemm", "score_gemm"):
+        assert per_seg[k] == (0.0, 0)
+    assert m.lib.sg_profile(m.h, 3) == 1          # SG_ERR_INVALID_ARG
+    m.close()
