@@ -166,8 +166,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm, AttnTcArgs a) {
   __shared__ __align__(8) uint64_t q_full;
   __shared__ __align__(8) uint64_t kv_full[ST], kv_empty[ST];
   __shared__ __align__(8) uint64_t s_full[NSB], p_full[NSB];
-  // o_full[g][i & 1] completes when the i-th P V of group g has landed
-  __shared__ __align__(8) uint64_t o_full[2][2];
   __shared__ float2 part_ml[2][QT];      // per group and row: (reference max, sum)
   __shared__ uint32_t tmem_slot;
   __shared__ int s_abort;
@@ -197,7 +195,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm, AttnTcArgs a) {
       tc::mbar_init(&s_full[b], 1);
       tc::mbar_init(&p_full[b], 4);
     }
-    for (int b = 0; b < 4; ++b) tc::mbar_init(&o_full[b >> 1][b & 1], 1);
     tc::fence_barrier_init();
     s_abort = 0;
   }
@@ -261,7 +258,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm, AttnTcArgs a) {
           tc::umma_bf16_ts(tmem + TM_O0 + (j & 1) * kDh, tmem + TM_S0 + b * KT + kk * 8, dv, idesc_o,
                            (j >= 2 || kk > 0) ? 1u : 0u);
         }
-        tc::umma_commit(&o_full[j & 1][(j >> 1) & 1]);
+        // one commit: it frees the K/V ring slot and tells the softmax group
+        // that P_j V_j has landed in its accumulator
         tc::umma_commit(&kv_empty[j % ST]);
         return true;
       };
@@ -281,15 +279,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm, AttnTcArgs a) {
     const uint32_t t_o = tl + TM_O0 + g * kDh;
     float m = -INFINITY, l = 0.f;                    // log2-domain reference max, running sum
     int k = 0;                                       // tiles this group has taken
-    int pv_seen = 0;                                 // completions of o_full[g] waited for
+    int pv_seen = 0;                                 // this group's P V products waited for
     bool ok = true;
-    // wait, in order, for this group's P V products up to count `upto`.  P V
-    // number i completes on o_full[g][i & 1]; a group waits for number i only
-    // after it has issued at most i + 2 of them, so neither barrier can be two
-    // phases ahead of the parity asked for
+    // wait, in order, for this group's P V products up to count `upto`.  Its
+    // product number i (tile t = g + 2 i) completes on the ring slot's
+    // kv_empty[t % ST]; the next completion of that slot is this group's
+    // product i + 3, and a group waits for number i only before it has written
+    // P number i + 2, so the barrier is never a phase ahead of the parity asked for
     auto wait_pv = [&](int upto) -> bool {
       for (; pv_seen < upto; ++pv_seen)
-        if (!warp_wait(&o_full[g][pv_seen & 1], (pv_seen >> 1) & 1, a.status)) return false;
+        if (!warp_wait(&kv_empty[(g + 2 * pv_seen) % ST], ((g + 2 * pv_seen) / ST) & 1, a.status)) return false;
       return true;
     };
     for (int j = g; j < ntiles; j += 2, ++k) {
