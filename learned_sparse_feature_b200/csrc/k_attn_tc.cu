@@ -233,10 +233,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm, AttnTcArgs a) {
       constexpr uint32_t idesc_o = tc::idesc_bf16_f32(QT, kDh, false, true);
       const uint64_t dq = tc::sdesc_k_sw128(base);
       bool ok = tc::mbar_wait(&q_full, 0, a.status, kErr);
-      auto issue_s = [&](int j) -> bool {
+      // A barrier probe by this thread between two batches of MMAs costs the
+      // tensor pipe about 80 cycles (measured), so each key tile's two waits
+      // (P_j ready, K/V of tile j+3 landed) are taken together before its batch.
+      auto wait_kv = [&](int j) -> bool {
+        return tc::mbar_wait(&kv_full[j % ST], (j / ST) & 1, a.status, kErr);
+      };
+      auto wait_p = [&](int j) -> bool {
+        return tc::mbar_wait(&p_full[j % NSB], (j / NSB) & 1, a.status, kErr);
+      };
+      auto issue_s = [&](int j) {
         const int st = j % ST, b = j % NSB;
-        if (!tc::mbar_wait(&kv_full[st], (j / ST) & 1, a.status, kErr)) return false;
-        tc::tc_fence_after();
         // buffer b last held P_{j-3}; P_{j-3} V_{j-3} was issued before this and
         // the tensor pipe runs this thread's MMAs in order
         const uint64_t dk = tc::sdesc_k_sw128(base + OFF_KV + st * STAGE_BYTES);
@@ -244,12 +251,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm, AttnTcArgs a) {
         for (int kk = 0; kk < kDh / 16; ++kk)
           tc::umma_bf16(tmem + TM_S0 + b * KT, dq + 2 * kk, dk + 2 * kk, idesc_s, kk > 0 ? 1u : 0u);
         tc::umma_commit(&s_full[b]);
-        return true;
       };
-      auto issue_pv = [&](int j) -> bool {
+      auto issue_pv = [&](int j) {
         const int b = j % NSB;
-        if (!tc::mbar_wait(&p_full[b], (j / NSB) & 1, a.status, kErr)) return false;
-        tc::tc_fence_after();
         const uint32_t vbase = base + OFF_KV + (j % ST) * STAGE_BYTES + KV_TILE;
 #pragma unroll
         for (int kk = 0; kk < KT / 16; ++kk) {
@@ -261,12 +265,19 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm, AttnTcArgs a) {
         // one commit: it frees the K/V ring slot and tells the softmax group
         // that P_j V_j has landed in its accumulator
         tc::umma_commit(&kv_empty[j % ST]);
-        return true;
       };
-      for (int j = 0; ok && j < NSB && j < ntiles; ++j) ok = issue_s(j);
+      for (int j = 0; ok && j < NSB && j < ntiles; ++j) {
+        ok = wait_kv(j);
+        tc::tc_fence_after();
+        if (ok) issue_s(j);
+      }
       for (int j = 0; ok && j < ntiles; ++j) {
-        ok = issue_pv(j);
-        if (ok && j + NSB < ntiles) ok = issue_s(j + NSB);
+        const bool more = j + NSB < ntiles;
+        ok = wait_p(j) && (!more || wait_kv(j + NSB));
+        tc::tc_fence_after();
+        if (!ok) break;
+        issue_pv(j);
+        if (more) issue_s(j + NSB);
       }
       pdl_trigger();                             // no more tensor work: the next kernel may start
       if (!ok) s_abort = 1;
