@@ -133,6 +133,12 @@ def make_weights(seed: int = 0, n_stages: int = N_STAGES, d: int = D,
     w["lg_bp"] = _bias(rng_h, d, d)
     w["lg_wz"] = _kaiming_uniform(rng_h, 1, d, gain_final_proj)[0]
     w["lg_bz"] = np.float32(_bias(rng_h, 1, d)[0])
+    # adaptive depth: one token-confidence classifier (linear + sigmoid) after
+    # every (self, cross) layer, from a third stream
+    rng_c = np.random.default_rng([seed, 2])
+    n_layers = n_stages // 2
+    w["tc_w"] = [_kaiming_uniform(rng_c, 1, d, 1.0)[0] for _ in range(n_layers)]
+    w["tc_b"] = [np.float32(_bias(rng_c, 1, d)[0]) for _ in range(n_layers)]
     return w
 
 

@@ -302,7 +302,80 @@ def double_softmax_head(x0, x1, Wp, bp, wz, bz):
     return double_softmax_log_assignment(sim, z0, z1), sim, z0, z1
 
 
+# --------------------------------------------------------------------------- adaptive depth
+def confidence_threshold(layer, n_layers):
+    """Per-layer exit threshold lambda_l = clip(0.8 + 0.1 exp(-4 l / L), 0, 1)
+    [LightGlue review, section 2.6 自适应深度, confidence_threshold].
+    Pinned by the two values the section prints (l = 1 and l = 9 of L = 9)."""
+    return float(np.clip(0.8 + 0.1 * math.exp(-4.0 * layer / n_layers), 0.0, 1.0))
+
+
+def token_confidence(x, w, b):
+    """Per-point confidence c_i = sigmoid(w . x_i + b) of the classifier after a
+    layer [LightGlue review, section 2.6: one confidence per point after every
+    layer but the last].  Reading: the classifier is one linear layer and a
+    sigmoid (the section's formula is garbled in the extracted text)."""
+    z = _as64(x) @ _as64(w) + float(b)
+    e = np.exp(-np.abs(z))                       # no overflow for large |z|
+    return np.where(z >= 0, 1.0 / (1.0 + e), e / (1.0 + e))
+
+
+def check_if_stop(confidences, layer, n_layers, depth_confidence, num_points):
+    """Stop after `layer` when the share of points whose confidence is not below
+    the layer's threshold exceeds depth_confidence (strict) [LightGlue review,
+    section 2.6, check_if_stop]: ratio = 1 - #(c < lambda_l) / num_points."""
+    lam = confidence_threshold(layer, n_layers)
+    ratio = 1.0 - float(np.sum(np.asarray(confidences) < lam)) / float(num_points)
+    return ratio > depth_confidence
+
+
+def attentional_gnn_adaptive(xs0, xs1, weights, heads, eps, depth_confidence, n_stages=None):
+    """The stages of attentional_gnn for a batch of pairs (lists of states), with
+    the adaptive-depth exit [LightGlue review, section 2.6]: a layer is one
+    (self, cross) pair of stages; after layer l < L - 1 the confidences of every
+    point of every pair decide one stop for the whole batch (reading: the
+    fraction is taken over all B (M + N) points; for B = 1 it is the pages'
+    num_points = m + n).  Returns (xs0, xs1, layers_run)."""
+    stages = weights["stages"]
+    if n_stages is None:
+        n_stages = len(stages)
+    n_layers = n_stages // 2
+    xs0, xs1 = list(xs0), list(xs1)
+    for layer in range(n_layers):
+        for s in (2 * layer, 2 * layer + 1):
+            for b in range(len(xs0)):
+                x0, x1 = xs0[b], xs1[b]
+                src0, src1 = (x1, x0) if s % 2 == 1 else (x0, x1)
+                d0 = attentional_propagation(x0, src0, stages[s], heads, eps)
+                d1 = attentional_propagation(x1, src1, stages[s], heads, eps)
+                xs0[b], xs1[b] = x0 + d0, x1 + d1
+        if layer == n_layers - 1 or depth_confidence is None or depth_confidence <= 0:
+            continue
+        conf = np.concatenate([token_confidence(np.concatenate([xs0[b], xs1[b]]),
+                                                weights["tc_w"][layer], weights["tc_b"][layer])
+                               for b in range(len(xs0))])
+        if check_if_stop(conf, layer, n_layers, depth_confidence, conf.size):
+            return xs0, xs1, layer + 1
+    return xs0, xs1, n_layers
+
+
 # --------------------------------------------------------------------------- whole pass
+def matching_head(x0, x1, weights, head="sinkhorn", iters=100, threshold=0.2):
+    """Score matrix + dustbin + log-Sinkhorn, or the double-softmax head, then the
+    mutual extraction, on the final GNN states of one pair."""
+    if head == "double_softmax":
+        logP, sim, z0, z1 = double_softmax_head(x0, x1, weights["lg_Wp"], weights["lg_bp"],
+                                                weights["lg_wz"], weights["lg_bz"])
+        m0, m1, s0, s1 = extract_matches(logP, threshold)
+        return {"log_P": logP, "matches0": m0, "matches1": m1, "mscores0": s0, "mscores1": s1,
+                "scores": sim, "z0": z0, "z1": z1}
+    S = score_matrix(x0, x1, weights["Wf"], weights["bf"])
+    logP = log_optimal_transport(S, float(weights["bin_score"]), iters)
+    m0, m1, s0, s1 = extract_matches(logP, threshold)
+    return {"log_P": logP, "matches0": m0, "matches1": m1, "mscores0": s0, "mscores1": s1,
+            "scores": S}
+
+
 def superglue_pair(kpts0, conf0, desc0, kpts1, conf1, desc1, weights,
                    img_w=640.0, img_h=480.0, heads=4, iters=100,
                    threshold=0.2, eps=1e-5, norm_mode=0, n_stages=None, head="sinkhorn"):
@@ -324,17 +397,23 @@ def superglue_pair(kpts0, conf0, desc0, kpts1, conf1, desc1, weights,
     x0 = keypoint_encoder(k0, conf0, desc0, weights, eps)
     x1 = keypoint_encoder(k1, conf1, desc1, weights, eps)
     x0, x1 = attentional_gnn(x0, x1, weights, heads, eps, n_stages)
-    if head == "double_softmax":
-        logP, sim, z0, z1 = double_softmax_head(x0, x1, weights["lg_Wp"], weights["lg_bp"],
-                                                weights["lg_wz"], weights["lg_bz"])
-        m0, m1, s0, s1 = extract_matches(logP, threshold)
-        return {"log_P": logP, "matches0": m0, "matches1": m1, "mscores0": s0, "mscores1": s1,
-                "scores": sim, "z0": z0, "z1": z1}
-    S = score_matrix(x0, x1, weights["Wf"], weights["bf"])
-    logP = log_optimal_transport(S, float(weights["bin_score"]), iters)
-    m0, m1, s0, s1 = extract_matches(logP, threshold)
-    return {"log_P": logP, "matches0": m0, "matches1": m1, "mscores0": s0, "mscores1": s1,
-            "scores": S}
+    return matching_head(x0, x1, weights, head, iters, threshold)
+
+
+def superglue_batch_adaptive(batch, weights, depth_confidence, img_w=640.0, img_h=480.0, heads=4,
+                             iters=100, threshold=0.2, eps=1e-5, norm_mode=0, n_stages=None,
+                             head="sinkhorn"):
+    """A whole batch (pairs of equal, non-zero M and N) with the adaptive-depth
+    exit decided over the batch; returns (list of per-pair results, layers run)."""
+    B = batch["kpts0"].shape[0]
+    xs0, xs1 = [], []
+    for b in range(B):
+        k0 = normalize_keypoints(batch["kpts0"][b], img_w, img_h, norm_mode)
+        k1 = normalize_keypoints(batch["kpts1"][b], img_w, img_h, norm_mode)
+        xs0.append(keypoint_encoder(k0, batch["conf0"][b], batch["desc0"][b], weights, eps))
+        xs1.append(keypoint_encoder(k1, batch["conf1"][b], batch["desc1"][b], weights, eps))
+    xs0, xs1, layers = attentional_gnn_adaptive(xs0, xs1, weights, heads, eps, depth_confidence, n_stages)
+    return [matching_head(xs0[b], xs1[b], weights, head, iters, threshold) for b in range(B)], layers
 
 
 def superglue_batch(batch, weights, pairs=None, **kw):

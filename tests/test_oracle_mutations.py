@@ -36,6 +36,12 @@ PIN_TESTS = [
     (pins.test_log_sigmoid_is_stable_and_complements, False),
     (pins.test_double_softmax_head_matches_torch_modules, True),
     (pins.test_double_softmax_recovers_a_planted_permutation, False),
+    (pins.test_confidence_threshold_printed_values, False),
+    (pins.test_check_if_stop_counts_strictly, False),
+    (pins.test_token_confidence_matches_torch_linear_sigmoid, False),
+    (pins.test_adaptive_gnn_that_never_stops_is_the_fixed_depth_gnn, True),
+    (pins.test_adaptive_gnn_stops_after_the_planted_layer, True),
+    (pins.test_adaptive_decision_pools_the_points_of_the_batch, True),
 ]
 
 
@@ -236,7 +242,56 @@ def _head_matchability_on_projection(x0, x1, Wp, bp, wz, bz):
     return O.double_softmax_log_assignment(sim, z0, z1), sim, z0, z1
 
 
+def _threshold_growing(layer, n_layers):
+    return float(np.clip(0.8 + 0.1 * math.exp(4.0 * layer / n_layers), 0.0, 1.0))
+
+
+def _stop_counts_equal_as_low(confidences, layer, n_layers, depth_confidence, num_points):
+    lam = O.confidence_threshold(layer, n_layers)
+    ratio = 1.0 - float(np.sum(np.asarray(confidences) <= lam)) / float(num_points)
+    return ratio > depth_confidence
+
+
+def _stop_at_equal_share(confidences, layer, n_layers, depth_confidence, num_points):
+    lam = O.confidence_threshold(layer, n_layers)
+    ratio = 1.0 - float(np.sum(np.asarray(confidences) < lam)) / float(num_points)
+    return ratio >= depth_confidence
+
+
+def _confidence_without_bias(x, w, b):
+    z = np.asarray(x, float) @ np.asarray(w, float)
+    return 1.0 / (1.0 + np.exp(-z))
+
+
+def _adaptive_last_pair_only(xs0, xs1, weights, heads, eps, depth_confidence, n_stages=None):
+    stages = weights["stages"]
+    n_stages = len(stages) if n_stages is None else n_stages
+    n_layers = n_stages // 2
+    xs0, xs1 = list(xs0), list(xs1)
+    for layer in range(n_layers):
+        for s in (2 * layer, 2 * layer + 1):
+            for b in range(len(xs0)):
+                x0, x1 = xs0[b], xs1[b]
+                src0, src1 = (x1, x0) if s % 2 == 1 else (x0, x1)
+                d0 = O.attentional_propagation(x0, src0, stages[s], heads, eps)
+                d1 = O.attentional_propagation(x1, src1, stages[s], heads, eps)
+                xs0[b], xs1[b] = x0 + d0, x1 + d1
+        if layer == n_layers - 1 or depth_confidence is None or depth_confidence <= 0:
+            continue
+        b = len(xs0) - 1
+        conf = O.token_confidence(np.concatenate([xs0[b], xs1[b]]), weights["tc_w"][layer],
+                                  weights["tc_b"][layer])
+        if O.check_if_stop(conf, layer, n_layers, depth_confidence, conf.size):
+            return xs0, xs1, layer + 1
+    return xs0, xs1, n_layers
+
+
 MUTATIONS = {
+    "exit threshold grows with depth": ("confidence_threshold", _threshold_growing),
+    "confidence at the threshold counted as low": ("check_if_stop", _stop_counts_equal_as_low),
+    "exit when the share equals depth_confidence": ("check_if_stop", _stop_at_equal_share),
+    "token confidence without its bias": ("token_confidence", _confidence_without_bias),
+    "exit decided on the last pair only": ("attentional_gnn_adaptive", _adaptive_last_pair_only),
     "double softmax over one axis twice": ("double_softmax_log_assignment", _dsm_same_axis_twice),
     "double softmax without certainties": ("double_softmax_log_assignment", _dsm_no_certainty),
     "double softmax dustbin sign": ("double_softmax_log_assignment", _dsm_dustbin_sign),

@@ -454,3 +454,98 @@ def test_double_softmax_recovers_a_planted_permutation():
     np.testing.assert_array_equal(m0, perm)
     np.testing.assert_array_equal(m1[perm], np.arange(4))
     assert np.all(s0 > 0.99)
+
+
+# --------------------------------------------------------------------------- adaptive depth
+def test_confidence_threshold_printed_values():
+    # the two thresholds the LightGlue review prints (section 2.6), to 3 decimals,
+    # and the l = 0 closed form 0.8 + 0.1
+    for row in _read_golden("confidence_threshold_lightglue.txt"):
+        _, layer, n_layers, value = row
+        assert abs(O.confidence_threshold(int(layer), int(n_layers)) - float(value)) < 5e-4
+    assert O.confidence_threshold(0, 9) == pytest.approx(0.9, abs=1e-15)
+    seq = [O.confidence_threshold(l, 9) for l in range(10)]
+    assert all(a > b for a, b in zip(seq, seq[1:]))
+
+
+def test_check_if_stop_counts_strictly():
+    lam = O.confidence_threshold(2, 9)
+    # 20 points: 19 at exactly the threshold (not below it: confident) and one below
+    conf = np.full(20, lam)
+    conf[3] = lam - 1e-9
+    assert O.check_if_stop(conf, 2, 9, 0.9, 20)          # ratio 0.95 > 0.9
+    assert not O.check_if_stop(conf, 2, 9, 0.95, 20)     # ratio 0.95 is not above 0.95
+    assert not O.check_if_stop(conf, 2, 9, 0.96, 20)
+    assert O.check_if_stop(np.full(5, 1.0), 8, 9, 0.99, 5)
+    assert not O.check_if_stop(np.full(5, 0.5), 0, 9, 0.0, 5)   # every point below 0.9
+
+
+def test_token_confidence_matches_torch_linear_sigmoid():
+    rng = np.random.default_rng(41)
+    x = rng.standard_normal((33, 256))
+    w = rng.standard_normal(256) * 0.1
+    b = 0.37
+    lin = torch.nn.Linear(256, 1).double()
+    with torch.no_grad():
+        lin.weight.copy_(torch.from_numpy(w)[None])
+        lin.bias.fill_(b)
+        ref = torch.sigmoid(lin(torch.from_numpy(x)))[:, 0].numpy()
+    np.testing.assert_allclose(O.token_confidence(x, w, b), ref, rtol=0, atol=1e-15)
+
+
+def _adaptive_inputs(weights, B=2, M=9, N=7, seed=5):
+    rng = np.random.default_rng(seed)
+    xs0 = [rng.standard_normal((M, 256)) for _ in range(B)]
+    xs1 = [rng.standard_normal((N, 256)) for _ in range(B)]
+    return xs0, xs1
+
+
+def test_adaptive_gnn_that_never_stops_is_the_fixed_depth_gnn(weights):
+    xs0, xs1 = _adaptive_inputs(weights)
+    # ratio > 1 is impossible: every layer runs
+    a0, a1, layers = O.attentional_gnn_adaptive(xs0, xs1, weights, 4, 1e-5, 1.0, n_stages=6)
+    assert layers == 3
+    for b in range(2):
+        r0, r1 = O.attentional_gnn(xs0[b], xs1[b], weights, 4, 1e-5, n_stages=6)
+        np.testing.assert_allclose(a0[b], r0, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(a1[b], r1, rtol=0, atol=1e-12)
+
+
+def test_adaptive_gnn_stops_after_the_planted_layer(weights):
+    xs0, xs1 = _adaptive_inputs(weights)
+    w = dict(weights)
+    w["tc_w"] = [np.zeros(256) for _ in range(9)]
+    for k in (0, 1, 2):
+        # classifiers certain "not confident" before layer k, "confident" at k
+        w["tc_b"] = [-50.0 if l < k else 50.0 for l in range(9)]
+        a0, a1, layers = O.attentional_gnn_adaptive(xs0, xs1, w, 4, 1e-5, 0.95, n_stages=8)
+        assert layers == k + 1
+        for b in range(2):
+            r0, r1 = O.attentional_gnn(xs0[b], xs1[b], w, 4, 1e-5, n_stages=2 * k + 2)
+            np.testing.assert_allclose(a0[b], r0, rtol=0, atol=1e-12)
+            np.testing.assert_allclose(a1[b], r1, rtol=0, atol=1e-12)
+    # no exit check after the last layer: a confident last layer changes nothing
+    w["tc_b"] = [-50.0, -50.0, -50.0, 50.0] + [50.0] * 5
+    assert O.attentional_gnn_adaptive(xs0, xs1, w, 4, 1e-5, 0.95, n_stages=8)[2] == 4
+
+
+def test_adaptive_decision_pools_the_points_of_the_batch(weights):
+    # pair 0's points all confident, pair 1's points all below the threshold
+    # (through the sign of one input channel): the pooled share is M0+N0 over
+    # all points, so the exit flips exactly where depth_confidence crosses it
+    w = dict(weights)
+    tw = np.zeros(256)
+    tw[0] = 100.0
+    w["tc_w"] = [tw] * 9
+    w["tc_b"] = [0.0] * 9
+    xs0, xs1 = _adaptive_inputs(weights, B=2, M=6, N=4)
+    xs0 = [np.abs(xs0[0]) + 50.0, -np.abs(xs0[1]) - 50.0]
+    xs1 = [np.abs(xs1[0]) + 50.0, -np.abs(xs1[1]) - 50.0]
+    # one stage pair changes the states, so look at the layer-0 confidences
+    # after the first layer, as the gnn does
+    a0, a1, _ = O.attentional_gnn_adaptive(xs0, xs1, w, 4, 1e-5, 1.0, n_stages=2)
+    conf = np.concatenate([O.token_confidence(np.concatenate([a0[b], a1[b]]), tw, 0.0) for b in range(2)])
+    share = 1.0 - np.mean(conf < O.confidence_threshold(0, 2))
+    assert 0.0 < share < 1.0
+    assert O.attentional_gnn_adaptive(xs0, xs1, w, 4, 1e-5, share - 1e-9, n_stages=4)[2] == 1
+    assert O.attentional_gnn_adaptive(xs0, xs1, w, 4, 1e-5, share, n_stages=4)[2] == 2
