@@ -103,6 +103,10 @@ typedef enum {
  *       (the similarity is <m0, m1> with m = (lg_Wp x + lg_bp) / D^(1/4)),
  *       matchability weights (D) and bias of z = lg_wz . x + lg_bz on the GNN
  *       states.  Wf, bf and bin_score are then not used.
+ *   tc_w[l], tc_b[l]: adaptive depth (only read when cfg.depth_confidence > 0):
+ *       the token-confidence classifier after layer l (stages 2l and 2l+1),
+ *       c = sigmoid(tc_w[l] . x + tc_b[l]) on each point's state, D weights;
+ *       needed for l < n_stages/2 - 1 (the LightGlue review, section 2.6).
  */
 typedef struct {
     const float* enc_W[SG_ENC_LAYERS];
@@ -127,6 +131,8 @@ typedef struct {
     const float* lg_bp;
     const float* lg_wz;
     float lg_bz;
+    const float* tc_w[SG_MAX_STAGES / 2];
+    float tc_b[SG_MAX_STAGES / 2];
 } sg_weights;
 
 /*
@@ -147,6 +153,11 @@ typedef struct {
     int norm_mode;
     int max_B, max_M, max_N;
     int head;                /* sg_head_t; the pages' LightGlue default threshold is 0.1 */
+    float depth_confidence;  /* adaptive depth: > 0 enables the exit after a (self, cross)
+                                layer l < L-1 when the share of points with confidence not
+                                below clip(0.8 + 0.1 exp(-4 l / L), 0, 1) exceeds it (one
+                                decision for the whole batch, over all B (M+N) points);
+                                <= 0 runs every stage.  Needs an even n_stages <= 32. */
 } sg_config;
 
 /* Create a handle on the current device: validates cfg, copies and packs the
@@ -212,6 +223,17 @@ sg_status_t sg_optimal_transport(sg_handle* h, int B, int M, int N,
  * reported an error.
  */
 sg_status_t sg_status(sg_handle* h, void* stream);
+
+/*
+ * Adaptive depth: synchronises `stream` and writes to *layers how many
+ * (self, cross) layers the last sg_match / sg_scores on this handle ran
+ * (ceil(n_stages / 2) when adaptive depth is off or no exit was taken).
+ * The skipped layers' kernels still launch and return at once; the final
+ * projection and the matching head run on the states at the exit.
+ * Returns SG_ERR_INVALID_ARG for a null pointer, SG_ERR_CUDA if the stream
+ * failed.
+ */
+sg_status_t sg_layers_run(sg_handle* h, int* layers, void* stream);
 
 /*
  * Step 5 of the double-softmax head on given inputs (the counterpart of

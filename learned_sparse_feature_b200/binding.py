@@ -26,7 +26,8 @@ STATUS = {0: "SG_OK", 1: "SG_ERR_INVALID_ARG", 2: "SG_ERR_SHAPE", 3: "SG_ERR_OOM
 EXPORTED = ["sg_create", "sg_destroy", "sg_match", "sg_match_host", "sg_scores",
             "sg_optimal_transport", "sg_status", "sg_strerror", "sg_launches_per_match",
             "sg_selftest_barrier_timeout", "sg_profile", "sg_profile_read",
-            "sg_optimal_transport_static", "sg_selftest_exp2_poly", "sg_assign_double_softmax"]
+            "sg_optimal_transport_static", "sg_selftest_exp2_poly", "sg_assign_double_softmax",
+            "sg_layers_run"]
 
 KERNEL_CLASSES = ["encoder", "qkv_gemm", "attention", "mlp1_gemm", "mlp2_gemm", "proj_gemm",
                   "score_gemm", "sinkhorn", "gnn"]
@@ -49,6 +50,7 @@ class SgWeights(C.Structure):
         ("Wf", _FP), ("bf", _FP),
         ("bin_score", C.c_float),
         ("lg_Wp", _FP), ("lg_bp", _FP), ("lg_wz", _FP), ("lg_bz", C.c_float),
+        ("tc_w", _FP * (SG_MAX_STAGES // 2)), ("tc_b", C.c_float * (SG_MAX_STAGES // 2)),
     ]
 
 
@@ -59,6 +61,7 @@ class SgConfig(C.Structure):
         ("img_w", C.c_float), ("img_h", C.c_float), ("norm_mode", C.c_int),
         ("max_B", C.c_int), ("max_M", C.c_int), ("max_N", C.c_int),
         ("head", C.c_int),
+        ("depth_confidence", C.c_float),
     ]
 
 
@@ -112,6 +115,8 @@ def load():
     lib.sg_profile_read.restype = i32
     lib.sg_optimal_transport_static.argtypes = [i32, i32, i32, vp, f32, i32, f32, vp, vp, vp, vp, vp, vp, vp]
     lib.sg_optimal_transport_static.restype = i32
+    lib.sg_layers_run.argtypes = [vp, C.POINTER(C.c_int), vp]
+    lib.sg_layers_run.restype = i32
     lib.sg_selftest_exp2_poly.argtypes = [vp, vp, i32, vp]
     lib.sg_selftest_exp2_poly.restype = i32
     _lib = lib
@@ -145,7 +150,7 @@ class Matcher:
     def __init__(self, weights: dict, max_B: int, max_M: int, max_N: int, precision: str = "bf16",
                  n_stages: int | None = None, sinkhorn_iters: int = 100, match_threshold: float = 0.2,
                  bn_eps: float = 1e-5, img_w: float = 640.0, img_h: float = 480.0, norm_mode: int = 0,
-                 head: str = "sinkhorn"):
+                 head: str = "sinkhorn", depth_confidence: float = -1.0):
         lib = load()
         self._keep = []
         w = SgWeights()
@@ -177,9 +182,13 @@ class Matcher:
             w.lg_bp = fp(weights["lg_bp"])
             w.lg_wz = fp(weights["lg_wz"])
             w.lg_bz = float(weights["lg_bz"])
+        if depth_confidence > 0:
+            for l in range(n // 2 - 1):
+                w.tc_w[l] = fp(weights["tc_w"][l])
+                w.tc_b[l] = float(weights["tc_b"][l])
         cfg = SgConfig(256, 4, n, sinkhorn_iters, match_threshold, bn_eps,
                        1 if precision == "bf16" else 0, img_w, img_h, norm_mode, max_B, max_M, max_N,
-                       HEADS[head])
+                       HEADS[head], depth_confidence)
         h = C.c_void_p()
         _check(lib.sg_create(C.byref(w), C.byref(cfg), C.byref(h)), "sg_create")
         self._keep = []
@@ -256,6 +265,12 @@ class Matcher:
         if self.lib.sg_profile_read(self.h, ms, cnt, n) < 0:
             raise SgError(4, "sg_profile_read")
         return {KERNEL_CLASSES[i]: (float(ms[i]), int(cnt[i])) for i in range(n)}
+
+    def layers_run(self, stream=None):
+        """(self, cross) layers the last pass ran (synchronises the stream)."""
+        n = C.c_int(0)
+        _check(self.lib.sg_layers_run(self.h, C.byref(n), _stream_ptr(stream)), "sg_layers_run")
+        return n.value
 
     def launches_per_match(self, B, M, N):
         return self.lib.sg_launches_per_match(self.h, B, M, N)

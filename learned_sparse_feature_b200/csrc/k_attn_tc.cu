@@ -67,6 +67,7 @@ struct AttnTcArgs {
   float scale_log2;
   float blind_limit;
   unsigned* status;
+  const unsigned* skip;   // adaptive depth: nothing to compute once *skip is set
 };
 
 __device__ __forceinline__ float fast_ex2(float x) {
@@ -205,8 +206,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm, AttnTcArgs a) {
   tc::tc_fence_after();
   const uint32_t tmem = tmem_slot;
   pdl_wait();                                    // q|k|v of the previous kernel are complete
+  // the adaptive-depth exit flag (written by an earlier kernel of the pass):
+  // once it is set no role does anything; all threads read it here
+  const bool skipped = a.skip != nullptr && *reinterpret_cast<const volatile unsigned*>(a.skip) != 0u;
 
-  if (warp == 8) {
+  if (skipped) {
+    if (warp == 9 && lane == 0) pdl_trigger();
+  } else if (warp == 8) {
     if (lane == 0) {
       // ---------------- TMA producer
       tc::mbar_arrive_expect_tx(&q_full, Q_BYTES);
@@ -439,7 +445,7 @@ cudaError_t launch_attention_tc(const AttnArgs& a, cudaStream_t s, unsigned* sta
     attr[emu] = true;
   }
   AttnTcArgs t{reinterpret_cast<__nv_bfloat16*>(a.msg), a.B, a.M, a.N, a.cross, a.scale_log2,
-               a.blind_limit > 0.f ? a.blind_limit : 18446744073709551616.f, status};
+               a.blind_limit > 0.f ? a.blind_limit : 18446744073709551616.f, status, a.skip};
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((nmax + QT - 1) / QT, kH, 2 * a.B);
   cfg.blockDim = dim3(kThreads);

@@ -52,6 +52,7 @@ struct TcArgs {
   float scale;
   unsigned* status;
   int b_const;           // W is constant (weights), not an output of an earlier kernel
+  const unsigned* skip;  // adaptive depth: nothing to compute once *skip is set
 };
 
 // Epilogue staging of one epilogue warp: one buffer set, a 32-row chunk of the
@@ -168,16 +169,24 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = tmem_slot;
+  // tiles this launch computes: none once the adaptive-depth exit flag, written
+  // by an earlier kernel of the pass, is set (every role reads it after its
+  // griddepcontrol.wait, so all see the same value)
+  int nt = ntiles;
+  auto exit_set = [&]() { return g.skip != nullptr && *reinterpret_cast<const volatile unsigned*>(g.skip) != 0u; };
   // the previous kernel's outputs must be complete before they are read and
   // before this kernel's outputs overwrite anything it still reads; the
   // producer first fetches constant weight tiles, which need neither
-  if (!(warp == 0 && lane == 0)) pdl_wait();
+  if (!(warp == 0 && lane == 0)) {
+    pdl_wait();
+    if (exit_set()) nt = 0;
+  }
 
   if (warp == 0) {
     if (lane == 0) {
       // ---------------- TMA producer
       int pre = 0;                               // ring stages whose W tile is already in flight
-      if (g.b_const && (int)blockIdx.x < ntiles) {
+      if (g.b_const && g.skip == nullptr && (int)blockIdx.x < ntiles) {
         const int t = blockIdx.x;
         const int tn = t % ntn, bz = t / (ntn * ntm);
         const int b_row = g.b_row0 + bz * g.b_batch_rows + tn * BN;
@@ -188,8 +197,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
         }
       }
       pdl_wait();
+      if (exit_set()) nt = 0;
       int it = 0;
-      for (int t = blockIdx.x; t < ntiles && !s_abort; t += gridDim.x) {
+      for (int t = blockIdx.x; t < nt && !s_abort; t += gridDim.x) {
         const int tn = t % ntn, tm = (t / ntn) % ntm, bz = t / (ntn * ntm);
         const int a_row = bz * g.a_batch_rows + tm * BM;
         const int b_row = g.b_row0 + bz * g.b_batch_rows + tn * BN;
@@ -218,7 +228,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
       constexpr uint32_t idesc = tc::idesc_bf16_f32(BM, BN);
       int it = 0, i = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++i) {
+      for (int t = blockIdx.x; t < nt && ok; t += gridDim.x, ++i) {
         const int b = i & 1;
         if (i >= 2 && !tc::mbar_wait(&tempty_bar[b], ((i >> 1) - 1) & 1, g.status, kErrGemmWait)) {
           ok = false;
@@ -266,7 +276,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
     uint32_t res_par = 0;                        // residual barrier parity
     bool res_pend = false;                       // a residual load issued and not yet waited for
     int i = 0;
-    for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++i) {
+    for (int t = blockIdx.x; t < nt; t += gridDim.x, ++i) {
       const int b = i & 1;
       const int tn = t % ntn, tm = (t / ntn) % ntm, bz = t / (ntn * ntm);
       const int n0 = tn * BN;
@@ -535,6 +545,7 @@ cudaError_t launch_gemm_tc(const GemmArgs& g, int epi, int batch, cudaStream_t s
   t.bias = g.bias; t.out = g.out; t.out2 = g.out2; t.ldo = g.ldo; t.strideO = g.strideO;
   t.scale = g.scale; t.status = status;
   t.b_const = g.w_dynamic ? 0 : 1;
+  t.skip = g.skip;
   // outputs: bf16 (bias epilogues), fp32 scores, fp32 residual stream + its bf16 copy
   CUtensorMap o, o2;
   const bool f32 = epi == EPI_SCALE || epi == EPI_RESIDUAL;

@@ -67,6 +67,12 @@ struct sg_handle {
   float score_scale;   // 1/sqrt(D) for the Sinkhorn head; 1 when folded into Wf (double softmax)
   float* lg_wz;        // double-softmax head: matchability weights (fp32) and bias
   float lg_bz;
+  // adaptive depth (cfg.depth_confidence > 0): per-layer token-confidence
+  // classifiers and the pass's stop / count words
+  bool adaptive;
+  float* tc_w[SG_MAX_STAGES / 2];
+  float tc_b[SG_MAX_STAGES / 2];
+  unsigned* depth_words;
   // workspace
   float* x32;
   __nv_bfloat16* x16;
@@ -268,6 +274,15 @@ sg_status_t pack_weights(sg_handle* h, const sg_weights* w) {
     h->alpha = w->bin_score;
     h->score_scale = (float)(1.0 / std::sqrt((double)D));
   }
+  if (h->adaptive) {
+    // one token-confidence classifier after every layer but the last
+    for (int l = 0; l + 1 < c.n_stages / 2; ++l) {
+      if (!w->tc_w[l]) return SG_ERR_INVALID_ARG;
+      std::vector<double> tw(w->tc_w[l], w->tc_w[l] + D);
+      h->tc_w[l] = upload_f32(h, tw, &ok);
+      h->tc_b[l] = w->tc_b[l];
+    }
+  }
   return ok ? SG_OK : SG_ERR_OOM;
 }
 
@@ -305,6 +320,12 @@ cudaError_t run_network(sg_handle* h, int B, int M, int N, const Inputs& in, flo
   ea.inv_scale = (float)(1.0 / (c.norm_mode == 0 ? 0.7 * (double)mx : 0.5 * (double)mx));
   mark(h, s, K_ENCODER);
   cudaError_t e;
+  // adaptive depth: clear the stop word and the per-layer counters of the pass
+  const unsigned* skip = nullptr;
+  if (h->adaptive) {
+    if ((e = cudaMemsetAsync(h->depth_words, 0, kDepthWords * sizeof(unsigned), s)) != cudaSuccess) return e;
+    skip = h->depth_words;
+  }
   if (h->use_tc) {
     // layers 0-2 on CUDA cores, layers 3-4 on the tensor cores
     __nv_bfloat16* h2 = reinterpret_cast<__nv_bfloat16*>(h->msg);   // R x 128, free until attention
@@ -336,6 +357,7 @@ cudaError_t run_network(sg_handle* h, int B, int M, int N, const Inputs& in, flo
     g.A0 = xin; g.A1 = nullptr; g.lda = kD; g.k_split = kD;
     g.W = w.Wqkv; g.bias = w.bqkv; g.out = h->qkv; g.ldo = kQKV;
     g.rows = R; g.cols = kQKV; g.K = kD; g.scale = 1.f;
+    g.skip = skip;
     if ((e = gemm(h, g, EPI_BIAS, h->bf16, 1, s, launches, K_QKV)) != cudaSuccess) return e;
     AttnArgs aa{};
     aa.qkv = h->qkv; aa.msg = h->msg; aa.B = B; aa.M = M; aa.N = N;
@@ -343,6 +365,7 @@ cudaError_t run_network(sg_handle* h, int B, int M, int N, const Inputs& in, flo
     aa.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)kDh));
     aa.exp_emu = h->attn_exp_emu;
     aa.blind_limit = h->attn_blind_limit;
+    aa.skip = skip;
     mark(h, s, K_ATTN);
     ++*launches;
     e = h->use_tc_attn ? launch_attention_tc(aa, s, h->status) : launch_attention_simt(aa, h->bf16, s);
@@ -352,13 +375,25 @@ cudaError_t run_network(sg_handle* h, int B, int M, int N, const Inputs& in, flo
     g.A0 = xin; g.A1 = h->msg; g.lda = kD; g.k_split = kD;
     g.W = w.W1; g.bias = w.b1; g.out = h->hid; g.ldo = 2 * kD;
     g.rows = R; g.cols = 2 * kD; g.K = 2 * kD; g.scale = 1.f;
+    g.skip = skip;
     if ((e = gemm(h, g, EPI_BIAS_RELU, h->bf16, 1, s, launches, K_MLP1)) != cudaSuccess) return e;
     // x += W2 h   (bias 0), refresh the bf16 shadow
     g = GemmArgs{};
     g.A0 = h->hid; g.A1 = nullptr; g.lda = 2 * kD; g.k_split = 2 * kD;
     g.W = w.W2; g.bias = nullptr; g.out = h->x32; g.out2 = h->x16; g.ldo = kD;
     g.rows = R; g.cols = kD; g.K = 2 * kD; g.scale = 1.f;
+    g.skip = skip;
     if ((e = gemm(h, g, EPI_RESIDUAL, h->bf16, 1, s, launches, K_MLP2)) != cudaSuccess) return e;
+    // adaptive depth: exit check after every (self, cross) layer but the last
+    // (LightGlue review, section 2.6); later GNN launches see its stop word
+    const int L = c.n_stages / 2, layer = st / 2;
+    if (h->adaptive && st % 2 == 1 && layer + 1 < L) {
+      const double lam = std::min(1.0, std::max(0.0, 0.8 + 0.1 * std::exp(-4.0 * layer / L)));
+      ++*launches;
+      if ((e = launch_depth_check(h->x32, R, h->tc_w[layer], h->tc_b[layer], (float)lam, c.depth_confidence,
+                                  layer, h->depth_words, s)) != cudaSuccess)
+        return e;
+    }
   }
   // f = Wf x + bf
   GemmArgs g{};
@@ -503,7 +538,8 @@ const char* sg_strerror(sg_status_t s) {
 int sg_launches_per_match(const sg_handle* h, int B, int M, int N) {
   if (!h || B == 0 || M == 0 || N == 0) return 0;
   const int net = (h->use_tc ? 5 : 3) + 4 * h->cfg.n_stages;   // encoder .. score GEMM
-  return net + (h->cfg.head == SG_HEAD_DOUBLE_SOFTMAX ? 7 : 1);  // matchability + 6 head kernels, or Sinkhorn
+  const int depth = h->adaptive ? h->cfg.n_stages / 2 - 1 : 0;  // exit checks
+  return net + depth + (h->cfg.head == SG_HEAD_DOUBLE_SOFTMAX ? 7 : 1);  // matchability + 6 head kernels, or Sinkhorn
 }
 
 sg_status_t sg_create(const sg_weights* w, const sg_config* cfg, sg_handle** out) {
@@ -518,6 +554,10 @@ sg_status_t sg_create(const sg_weights* w, const sg_config* cfg, sg_handle** out
       (cfg->head != SG_HEAD_SINKHORN && cfg->head != SG_HEAD_DOUBLE_SOFTMAX))
     return SG_ERR_INVALID_ARG;
   if (cfg->max_N > sinkhorn_max_columns()) return SG_ERR_UNSUPPORTED;   // transport kernel columns
+  if (std::isnan(cfg->depth_confidence)) return SG_ERR_INVALID_ARG;
+  // adaptive depth works on whole (self, cross) layers
+  if (cfg->depth_confidence > 0.f && (cfg->n_stages % 2 != 0 || cfg->n_stages / 2 > 16))
+    return SG_ERR_UNSUPPORTED;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return SG_ERR_UNSUPPORTED; }
   cudaDeviceProp prop;
@@ -529,6 +569,7 @@ sg_status_t sg_create(const sg_weights* w, const sg_config* cfg, sg_handle** out
   h->device = dev;
   h->num_sms = prop.multiProcessorCount;
   h->bf16 = cfg->precision == SG_PRECISION_BF16;
+  h->adaptive = cfg->depth_confidence > 0.f;
   h->use_tc = h->bf16 && tc_available() && std::getenv("SG_FORCE_SIMT") == nullptr;
   h->use_tc_attn = h->use_tc && std::getenv("SG_SIMT_ATTENTION") == nullptr;
   {
@@ -570,6 +611,7 @@ sg_status_t sg_create(const sg_weights* w, const sg_config* cfg, sg_handle** out
   h->z0 = (float*)al(Bm * Mm * 4);
   h->z1 = (float*)al(Bm * Nm * 4);
   h->status = (unsigned*)al(sizeof(unsigned));
+  h->depth_words = (unsigned*)al(kDepthWords * sizeof(unsigned));
   h->s_k0 = (float*)al(Bm * Mm * 2 * 4);
   h->s_c0 = (float*)al(Bm * Mm * 4);
   h->s_d0 = (float*)al(Bm * Mm * kD * 4);
@@ -787,6 +829,21 @@ int sg_profile_read(sg_handle* h, float* ms_by_class, int* launches_by_class, in
     if (c >= 0 && c < n_classes) { ms_by_class[c] += ms; launches_by_class[c] += 1; }
   }
   return n_classes;
+}
+
+sg_status_t sg_layers_run(sg_handle* h, int* layers, void* stream) {
+  if (!h || !layers) return SG_ERR_INVALID_ARG;
+  const int all = (h->cfg.n_stages + 1) / 2;
+  if (!h->adaptive) {
+    *layers = all;
+    return SG_OK;
+  }
+  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+  unsigned w[2] = {0u, 0u};
+  if (e == cudaSuccess) e = cudaMemcpy(w, h->depth_words, sizeof(w), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_err(h, e);
+  *layers = w[0] ? (int)w[1] : all;
+  return SG_OK;
 }
 
 sg_status_t sg_status(sg_handle* h, void* stream) {

@@ -45,6 +45,7 @@ struct GemmArgs {
   long long strideA, strideW, strideO;
   float scale;
   int w_dynamic;   // W is written by an earlier kernel of the pass (the score GEMM's f_B), not a weight
+  const unsigned* skip;   // adaptive depth: when *skip != 0 (set by an earlier kernel) the launch does nothing
 };
 
 // Attention over the stacked state of B pairs: rows [b*P, b*P+M) are image A of
@@ -58,6 +59,7 @@ struct AttnArgs {
   float scale_log2;   // log2(e) / sqrt(d_head)
   int exp_emu;        // tensor-core path: of every 8 exp2 pairs, how many use the FMA pipe (0, 2, 3 or 4)
   float blind_limit;  // tensor-core path: bound on a key tile's sum of 2^(s - m) before the row's max is renewed
+  const unsigned* skip;   // adaptive depth: when *skip != 0 (set by an earlier kernel) the launch does nothing
 };
 
 struct EncArgs {
@@ -114,6 +116,16 @@ cudaError_t sinkhorn_prepare(int num_sms);   // kernel attributes (called once, 
 int sinkhorn_max_columns();                  // largest N the transport kernel supports
 size_t sinkhorn_scratch_bytes(int B, int M, int N);
 size_t sinkhorn_acc_floats_per_buffer(int N);   // column accumulator floats per (pair, rotation)
+// Adaptive depth (k_depth.cu): after layer `layer`, count the points of the
+// rows x 256 fp32 states x32 whose confidence sigmoid(w . x + b) is below
+// lambda; the last block to finish sets words[0] = 1 (stop) and words[1] =
+// layer + 1 when 1 - low / rows > depth_conf.  words: [stop, layers run,
+// low count per layer (16), finished blocks per layer (16)], zeroed per pass.
+// Does nothing when words[0] is already set.
+constexpr int kDepthWords = 2 + 2 * 16;
+cudaError_t launch_depth_check(const float* x32, int rows, const float* w, float b, float lambda,
+                               float depth_conf, int layer, unsigned* words, cudaStream_t s);
+
 // Double-softmax matching head (k_dsm.cu).
 size_t dsm_scratch_bytes(int B, int M, int N);
 cudaError_t launch_dsm_matchability(const float* x32, int B, int M, int N, const float* wz, float bz, float* z0,
