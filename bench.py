@@ -254,7 +254,7 @@ def run_reference(args, w):
     }
 
 
-def _config(w, n_gpus, head="sinkhorn"):
+def _config(w, n_gpus, head="sinkhorn", exit_layer=None):
     c = {"workload": w.name, "B_per_gpu": w.B, "M": w.M, "N": w.N, "stages": synth.N_STAGES,
          "sinkhorn_iters": synth.SINKHORN_ITERS, "precision": w.precision,
          "parallelism": f"replicas{n_gpus}", "l2": "flushed (256 MiB write) before every timed step"}
@@ -262,7 +262,23 @@ def _config(w, n_gpus, head="sinkhorn"):
         c["head"] = head
         c["match_threshold"] = DSM_THRESHOLD
         del c["sinkhorn_iters"]
+    if exit_layer is not None:
+        c["adaptive_depth"] = {"depth_confidence": EXIT_DEPTH_CONFIDENCE, "exit_after_layer": exit_layer,
+                               "classifier": "planted: confidences 0 before the layer, 1 at it"}
     return c
+
+
+EXIT_DEPTH_CONFIDENCE = 0.95
+
+
+def planted_exit_weights(weights, exit_layer):
+    """Token-confidence classifiers that make the adaptive-depth exit happen
+    after `exit_layer` (random-init weights give no meaningful confidences)."""
+    w = dict(weights)
+    n_layers = len(weights["tc_w"])
+    w["tc_w"] = [np.zeros_like(weights["tc_w"][0]) for _ in range(n_layers)]
+    w["tc_b"] = [np.float32(-30.0 if l < exit_layer else 30.0) for l in range(n_layers)]
+    return w
 
 
 def run_native(args, w):
@@ -287,13 +303,17 @@ def run_native(args, w):
     cpu_baseline = None
     weights = synth.make_weights(0)
     batch = synth.make_batch(w, shard_pairs(B, rank), B)
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    exit_layer = args.exit_layer
+    if exit_layer is not None:
+        weights = planted_exit_weights(weights, exit_layer)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and exit_layer is None:
         t, desc = oracle_step(batch, weights, head=args.head)
         cpu_baseline = {"value": 1.0 / t, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle", "sample": desc}
 
     dsm = args.head == "double_softmax"
     m = Matcher(weights, B, M, N, precision=w.precision, head=args.head,
-                match_threshold=DSM_THRESHOLD if dsm else synth.MATCH_THRESHOLD)
+                match_threshold=DSM_THRESHOLD if dsm else synth.MATCH_THRESHOLD,
+                depth_confidence=EXIT_DEPTH_CONFIDENCE if exit_layer is not None else -1.0)
     t = {k: torch.from_numpy(np.ascontiguousarray(batch[k])).to(dev)
          for k in ("kpts0", "conf0", "desc0", "kpts1", "conf1", "desc1")}
     logP = torch.empty((B, M + 1, N + 1), dtype=torch.float32, device=dev)
@@ -451,7 +471,7 @@ def run_native(args, w):
         "vs_baseline": (value / PAGES_PAIRS_PER_S[w.name]) if w.name in PAGES_PAIRS_PER_S else None,
         "dtype": "bf16" if w.precision == "bf16" else "f32",
         "data": "synthetic (seeded keypoint pairs, random-init weights)",
-        "config": _config(w, world, args.head),
+        "config": _config(w, world, args.head, exit_layer),
         "roofline": roofline,
         "gnn_tensor_frac": gnn_segment["frac_tensor"] if gnn_segment else None,
         "gnn": gnn_segment,
@@ -465,6 +485,10 @@ def run_native(args, w):
         "clocks": clk,
         "cpu_baseline": cpu_baseline,
     }
+    if exit_layer is not None:
+        # layers run by the last pass; the skipped layers' kernels still launch
+        # (and return at once), so gpu_launches counts them
+        out["layers_run"] = m.layers_run(stream)
     m.close()
     return out if rank == 0 else None
 
@@ -480,6 +504,9 @@ def main():
     ap.add_argument("--head", default="sinkhorn", choices=["sinkhorn", "double_softmax"],
                     help="matching head: dustbin + Sinkhorn (the default, the headline metric) or "
                          "the double-softmax head")
+    ap.add_argument("--exit-layer", type=int, default=None,
+                    help="adaptive depth with classifiers planted so that the pass exits after this "
+                         "(self, cross) layer (0-based; synthetic, no CPU baseline)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

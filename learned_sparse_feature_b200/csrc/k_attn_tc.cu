@@ -160,7 +160,9 @@ __device__ __forceinline__ float exp_row(const float (&s)[KT], float scale, floa
   return (a0 + a1) + (b0 + b1);
 }
 
-template <int EMU>
+// SKIP: the launch reads the adaptive-depth exit flag (a separate instantiation,
+// so the launches of a pass without adaptive depth run the kernel without it).
+template <int EMU, bool SKIP>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tm, AttnTcArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -208,7 +210,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm, AttnTcArgs a) {
   pdl_wait();                                    // q|k|v of the previous kernel are complete
   // the adaptive-depth exit flag (written by an earlier kernel of the pass):
   // once it is set no role does anything; all threads read it here
-  const bool skipped = a.skip != nullptr && *reinterpret_cast<const volatile unsigned*>(a.skip) != 0u;
+  bool skipped = false;
+  if constexpr (SKIP) skipped = *reinterpret_cast<const volatile unsigned*>(a.skip) != 0u;
 
   if (skipped) {
     if (warp == 9 && lane == 0) pdl_trigger();
@@ -436,13 +439,16 @@ cudaError_t launch_attention_tc(const AttnArgs& a, cudaStream_t s, unsigned* sta
   // share of the exponentials taken on the FMA pipe: exp_emu of every 8 pairs
   const int emu = (a.exp_emu == 2 || a.exp_emu == 3 || a.exp_emu == 4) ? a.exp_emu : 0;
   using Kern = void (*)(const CUtensorMap, AttnTcArgs);
-  Kern kern = emu == 0 ? attn_tc_kernel<0> : emu == 2 ? attn_tc_kernel<2> : emu == 4 ? attn_tc_kernel<4>
-                                                                                 : attn_tc_kernel<3>;
-  static bool attr[5] = {};
-  if (!attr[emu]) {
+  const bool sk = a.skip != nullptr;
+  Kern kern = sk ? (emu == 0 ? attn_tc_kernel<0, true> : emu == 2 ? attn_tc_kernel<2, true>
+                    : emu == 4 ? attn_tc_kernel<4, true> : attn_tc_kernel<3, true>)
+                 : (emu == 0 ? attn_tc_kernel<0, false> : emu == 2 ? attn_tc_kernel<2, false>
+                    : emu == 4 ? attn_tc_kernel<4, false> : attn_tc_kernel<3, false>);
+  static bool attr[2][5] = {};
+  if (!attr[sk][emu]) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    attr[emu] = true;
+    attr[sk][emu] = true;
   }
   AttnTcArgs t{reinterpret_cast<__nv_bfloat16*>(a.msg), a.B, a.M, a.N, a.cross, a.scale_log2,
                a.blind_limit > 0.f ? a.blind_limit : 18446744073709551616.f, status, a.skip};

@@ -113,8 +113,10 @@ __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.lau
 // ordered (batch, row tile, column tile) with the column tile fastest so
 // consecutive CTAs share the A tile in L2.  The accumulator is double-buffered
 // in TMEM: the epilogue warps drain tile i while the MMA warp accumulates tile
-// i + 1.
-template <int BN, int EPI>
+// i + 1.  SKIP: the launch reads the adaptive-depth exit flag (a separate
+// instantiation, so the launches of a pass without adaptive depth run the
+// kernel without any of it).
+template <int BN, int EPI, bool SKIP>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
                const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmO,
@@ -173,20 +175,22 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
   // by an earlier kernel of the pass, is set (every role reads it after its
   // griddepcontrol.wait, so all see the same value)
   int nt = ntiles;
-  auto exit_set = [&]() { return g.skip != nullptr && *reinterpret_cast<const volatile unsigned*>(g.skip) != 0u; };
+  auto exit_set = [&]() { return *reinterpret_cast<const volatile unsigned*>(g.skip) != 0u; };
   // the previous kernel's outputs must be complete before they are read and
   // before this kernel's outputs overwrite anything it still reads; the
   // producer first fetches constant weight tiles, which need neither
   if (!(warp == 0 && lane == 0)) {
     pdl_wait();
-    if (exit_set()) nt = 0;
+    if constexpr (SKIP) {
+      if (exit_set()) nt = 0;
+    }
   }
 
   if (warp == 0) {
     if (lane == 0) {
       // ---------------- TMA producer
       int pre = 0;                               // ring stages whose W tile is already in flight
-      if (g.b_const && g.skip == nullptr && (int)blockIdx.x < ntiles) {
+      if (g.b_const && !SKIP && (int)blockIdx.x < ntiles) {
         const int t = blockIdx.x;
         const int tn = t % ntn, bz = t / (ntn * ntm);
         const int b_row = g.b_row0 + bz * g.b_batch_rows + tn * BN;
@@ -197,7 +201,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
         }
       }
       pdl_wait();
-      if (exit_set()) nt = 0;
+      if constexpr (SKIP) {
+        if (exit_set()) nt = 0;
+      }
       int it = 0;
       for (int t = blockIdx.x; t < nt && !s_abort; t += gridDim.x) {
         const int tn = t % ntn, tm = (t / ntn) % ntm, bz = t / (ntn * ntm);
@@ -457,10 +463,10 @@ bool make_out_map(CUtensorMap* m, void* ptr, bool f32, long long rows, long long
   return r == CUDA_SUCCESS;
 }
 
-template <int BN, int EPI>
+template <int BN, int EPI, bool SKIP>
 cudaError_t launch_t(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b, const CUtensorMap& o,
                      const CUtensorMap& o2, const TcArgs& t, int grid, cudaStream_t s) {
-  auto kern = gemm_tc_kernel<BN, EPI>;
+  auto kern = gemm_tc_kernel<BN, EPI, SKIP>;
   constexpr int smem = Smem<BN, EPI>::BYTES;
   static bool attr = false;
   if (!attr) {
@@ -481,15 +487,23 @@ cudaError_t launch_t(const CUtensorMap& a0, const CUtensorMap& a1, const CUtenso
   return cudaLaunchKernelEx(&cfg, kern, a0, a1, b, o, o2, t);
 }
 
-template <int BN>
+template <int BN, bool SKIP>
 cudaError_t launch_epi(int epi, const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b,
                        const CUtensorMap& o, const CUtensorMap& o2, const TcArgs& t, int grid, cudaStream_t s) {
   switch (epi) {
-    case EPI_BIAS: return launch_t<BN, EPI_BIAS>(a0, a1, b, o, o2, t, grid, s);
-    case EPI_BIAS_RELU: return launch_t<BN, EPI_BIAS_RELU>(a0, a1, b, o, o2, t, grid, s);
-    case EPI_RESIDUAL: return launch_t<BN, EPI_RESIDUAL>(a0, a1, b, o, o2, t, grid, s);
-    default: return launch_t<BN, EPI_SCALE>(a0, a1, b, o, o2, t, grid, s);
+    case EPI_BIAS: return launch_t<BN, EPI_BIAS, SKIP>(a0, a1, b, o, o2, t, grid, s);
+    case EPI_BIAS_RELU: return launch_t<BN, EPI_BIAS_RELU, SKIP>(a0, a1, b, o, o2, t, grid, s);
+    case EPI_RESIDUAL: return launch_t<BN, EPI_RESIDUAL, SKIP>(a0, a1, b, o, o2, t, grid, s);
+    default: return launch_t<BN, EPI_SCALE, SKIP>(a0, a1, b, o, o2, t, grid, s);
   }
+}
+
+template <int BN>
+cudaError_t launch_bn(int epi, const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b,
+                      const CUtensorMap& o, const CUtensorMap& o2, const TcArgs& t, int grid, cudaStream_t s) {
+  // the exit-flag instantiations only for launches that carry the flag
+  return t.skip ? launch_epi<BN, true>(epi, a0, a1, b, o, o2, t, grid, s)
+                : launch_epi<BN, false>(epi, a0, a1, b, o, o2, t, grid, s);
 }
 
 }  // namespace
@@ -558,10 +572,10 @@ cudaError_t launch_gemm_tc(const GemmArgs& g, int epi, int batch, cudaStream_t s
   const long long tiles = row_tiles * ((g.cols + BN - 1) / BN);
   const int grid = (int)(tiles < nsm ? tiles : nsm);
   switch (BN) {
-    case 256: return launch_epi<256>(epi, a0, a1, b, o, o2, t, grid, s);
-    case 192: return launch_epi<192>(epi, a0, a1, b, o, o2, t, grid, s);
-    case 128: return launch_epi<128>(epi, a0, a1, b, o, o2, t, grid, s);
-    default: return launch_epi<64>(epi, a0, a1, b, o, o2, t, grid, s);
+    case 256: return launch_bn<256>(epi, a0, a1, b, o, o2, t, grid, s);
+    case 192: return launch_bn<192>(epi, a0, a1, b, o, o2, t, grid, s);
+    case 128: return launch_bn<128>(epi, a0, a1, b, o, o2, t, grid, s);
+    default: return launch_bn<64>(epi, a0, a1, b, o, o2, t, grid, s);
   }
 }
 
