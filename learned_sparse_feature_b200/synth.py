@@ -139,6 +139,10 @@ def make_weights(seed: int = 0, n_stages: int = N_STAGES, d: int = D,
     n_layers = n_stages // 2
     w["tc_w"] = [_kaiming_uniform(rng_c, 1, d, 1.0)[0] for _ in range(n_layers)]
     w["tc_b"] = [np.float32(_bias(rng_c, 1, d)[0]) for _ in range(n_layers)]
+    # point pruning: the matchability of every layer's assignment head, a fourth stream
+    rng_m = np.random.default_rng([seed, 3])
+    w["mt_w"] = [_kaiming_uniform(rng_m, 1, d, 1.0)[0] for _ in range(n_layers)]
+    w["mt_b"] = [np.float32(_bias(rng_m, 1, d)[0]) for _ in range(n_layers)]
     return w
 
 

@@ -313,8 +313,8 @@ def confidence_threshold(layer, n_layers):
 def token_confidence(x, w, b):
     """Per-point confidence c_i = sigmoid(w . x_i + b) of the classifier after a
     layer [LightGlue review, section 2.6: one confidence per point after every
-    layer but the last].  Reading: the classifier is one linear layer and a
-    sigmoid (the section's formula is garbled in the extracted text)."""
+    layer but the last; section 2.5: the classifier is a linear layer and a
+    sigmoid on the layer's state]."""
     z = _as64(x) @ _as64(w) + float(b)
     e = np.exp(-np.abs(z))                       # no overflow for large |z|
     return np.where(z >= 0, 1.0 / (1.0 + e), e / (1.0 + e))
@@ -329,19 +329,39 @@ def check_if_stop(confidences, layer, n_layers, depth_confidence, num_points):
     return ratio > depth_confidence
 
 
-def attentional_gnn_adaptive(xs0, xs1, weights, heads, eps, depth_confidence, n_stages=None):
+def attentional_gnn_adaptive(xs0, xs1, weights, heads, eps, depth_confidence, n_stages=None,
+                             width_confidence=None, pruning_threshold=1536):
     """The stages of attentional_gnn for a batch of pairs (lists of states), with
-    the adaptive-depth exit [LightGlue review, section 2.6]: a layer is one
-    (self, cross) pair of stages; after layer l < L - 1 the confidences of every
-    point of every pair decide one stop for the whole batch (reading: the
-    fraction is taken over all B (M + N) points; for B = 1 it is the pages'
-    num_points = m + n).  Returns (xs0, xs1, layers_run)."""
+    the adaptive-depth exit [LightGlue review, section 2.6] and, when
+    width_confidence > 0, point pruning [section 2.7].  A layer is one (self,
+    cross) pair of stages.  After layer l < L - 1:
+
+    * exit: the confidences of every remaining point of every pair decide one
+      stop for the whole batch; the share is 1 - #(c < lambda_l) / num_points
+      with num_points the original point count (the listing passes m + n, so a
+      pruned point counts as confident).  Reading: for a batch, num_points is
+      all B (M + N) original points; for B = 1 it is the pages' m + n.
+    * pruning (if the run goes on): each image of each pair with more than
+      pruning_threshold remaining points keeps the points that
+      get_pruning_mask keeps (matchability from the layer's head,
+      weights["mt_w"][l], weights["mt_b"][l]; confidences only when the exit
+      is enabled); the others leave every later layer (as queries and keys).
+
+    Returns (xs0, xs1, kept0, kept1, layers_run); kept* are the original
+    indices of the points still present, in order."""
     stages = weights["stages"]
     if n_stages is None:
         n_stages = len(stages)
     n_layers = n_stages // 2
+    depth = depth_confidence is not None and depth_confidence > 0
+    width = width_confidence is not None and width_confidence > 0
     xs0, xs1 = list(xs0), list(xs1)
+    kept0 = [np.arange(len(x)) for x in xs0]
+    kept1 = [np.arange(len(x)) for x in xs1]
+    num_points = sum(len(x) for x in xs0) + sum(len(x) for x in xs1)
     for layer in range(n_layers):
+        if any(len(x) == 0 for x in xs0) or any(len(x) == 0 for x in xs1):
+            break                                # a pair without points left: no more layers
         for s in (2 * layer, 2 * layer + 1):
             for b in range(len(xs0)):
                 x0, x1 = xs0[b], xs1[b]
@@ -349,14 +369,43 @@ def attentional_gnn_adaptive(xs0, xs1, weights, heads, eps, depth_confidence, n_
                 d0 = attentional_propagation(x0, src0, stages[s], heads, eps)
                 d1 = attentional_propagation(x1, src1, stages[s], heads, eps)
                 xs0[b], xs1[b] = x0 + d0, x1 + d1
-        if layer == n_layers - 1 or depth_confidence is None or depth_confidence <= 0:
-            continue
-        conf = np.concatenate([token_confidence(np.concatenate([xs0[b], xs1[b]]),
-                                                weights["tc_w"][layer], weights["tc_b"][layer])
-                               for b in range(len(xs0))])
-        if check_if_stop(conf, layer, n_layers, depth_confidence, conf.size):
-            return xs0, xs1, layer + 1
-    return xs0, xs1, n_layers
+        if layer == n_layers - 1:
+            continue                             # no exit and no pruning after the last layer
+        conf0 = conf1 = None
+        if depth:
+            conf0 = [token_confidence(x, weights["tc_w"][layer], weights["tc_b"][layer]) for x in xs0]
+            conf1 = [token_confidence(x, weights["tc_w"][layer], weights["tc_b"][layer]) for x in xs1]
+            if check_if_stop(np.concatenate(conf0 + conf1), layer, n_layers, depth_confidence, num_points):
+                return xs0, xs1, kept0, kept1, layer + 1
+        if width:
+            for b in range(len(xs0)):
+                for xs, kept, conf in ((xs0, kept0, conf0), (xs1, kept1, conf1)):
+                    if len(xs[b]) <= pruning_threshold:
+                        continue
+                    scores = matchability(xs[b], weights["mt_w"][layer], weights["mt_b"][layer])
+                    keep = get_pruning_mask(None if conf is None else conf[b], scores, layer, n_layers,
+                                            width_confidence)
+                    xs[b], kept[b] = xs[b][keep], kept[b][keep]
+    return xs0, xs1, kept0, kept1, n_layers
+
+
+def matchability(x, w, b):
+    """sigmoid(w . x + b): the matchability of the layer's assignment head
+    [LightGlue review, section 2.4, MatchAssignment.get_matchability]."""
+    z = _as64(x) @ _as64(w) + float(b)
+    e = np.exp(-np.abs(z))
+    return np.where(z >= 0, 1.0 / (1.0 + e), e / (1.0 + e))
+
+
+def get_pruning_mask(confidences, scores, layer, n_layers, width_confidence):
+    """Points kept for the next layer: matchability above 1 - width_confidence,
+    and every point whose confidence is not above the layer's threshold (an
+    uncertain point is never pruned) [LightGlue review, section 2.7,
+    get_pruning_mask]."""
+    keep = np.asarray(scores) > (1.0 - width_confidence)
+    if confidences is not None:
+        keep = keep | (np.asarray(confidences) <= confidence_threshold(layer, n_layers))
+    return keep
 
 
 # --------------------------------------------------------------------------- whole pass
@@ -402,9 +451,14 @@ def superglue_pair(kpts0, conf0, desc0, kpts1, conf1, desc1, weights,
 
 def superglue_batch_adaptive(batch, weights, depth_confidence, img_w=640.0, img_h=480.0, heads=4,
                              iters=100, threshold=0.2, eps=1e-5, norm_mode=0, n_stages=None,
-                             head="sinkhorn"):
+                             head="sinkhorn", width_confidence=None, pruning_threshold=1536):
     """A whole batch (pairs of equal, non-zero M and N) with the adaptive-depth
-    exit decided over the batch; returns (list of per-pair results, layers run)."""
+    exit decided over the batch and optional point pruning; returns (list of
+    per-pair results, layers run).  With pruning, the head runs on the points
+    left after the last layer and its matches are mapped back to the original
+    indices [LightGlue review, section 2.7: prune0/prune1 and the map back];
+    a pruned point is unmatched (-1, score 0); log_P covers the points left,
+    listed in "kept0" / "kept1"."""
     B = batch["kpts0"].shape[0]
     xs0, xs1 = [], []
     for b in range(B):
@@ -412,8 +466,27 @@ def superglue_batch_adaptive(batch, weights, depth_confidence, img_w=640.0, img_
         k1 = normalize_keypoints(batch["kpts1"][b], img_w, img_h, norm_mode)
         xs0.append(keypoint_encoder(k0, batch["conf0"][b], batch["desc0"][b], weights, eps))
         xs1.append(keypoint_encoder(k1, batch["conf1"][b], batch["desc1"][b], weights, eps))
-    xs0, xs1, layers = attentional_gnn_adaptive(xs0, xs1, weights, heads, eps, depth_confidence, n_stages)
-    return [matching_head(xs0[b], xs1[b], weights, head, iters, threshold) for b in range(B)], layers
+    M, N = len(xs0[0]), len(xs1[0])
+    xs0, xs1, kept0, kept1, layers = attentional_gnn_adaptive(
+        xs0, xs1, weights, heads, eps, depth_confidence, n_stages, width_confidence, pruning_threshold)
+    out = []
+    for b in range(B):
+        m0 = np.full(M, -1, np.int32)
+        m1 = np.full(N, -1, np.int32)
+        s0 = np.zeros(M, F64)
+        s1 = np.zeros(N, F64)
+        res = {"log_P": None, "kept0": kept0[b], "kept1": kept1[b]}
+        if len(kept0[b]) and len(kept1[b]):
+            r = matching_head(xs0[b], xs1[b], weights, head, iters, threshold)
+            sub0, sub1 = r["matches0"], r["matches1"]
+            m0[kept0[b]] = np.where(sub0 >= 0, kept1[b][np.maximum(sub0, 0)], -1)
+            m1[kept1[b]] = np.where(sub1 >= 0, kept0[b][np.maximum(sub1, 0)], -1)
+            s0[kept0[b]] = r["mscores0"]
+            s1[kept1[b]] = r["mscores1"]
+            res.update({k: v for k, v in r.items() if k not in ("matches0", "matches1", "mscores0", "mscores1")})
+        res.update({"matches0": m0, "matches1": m1, "mscores0": s0, "mscores1": s1})
+        out.append(res)
+    return out, layers
 
 
 def superglue_batch(batch, weights, pairs=None, **kw):

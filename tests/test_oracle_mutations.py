@@ -42,6 +42,12 @@ PIN_TESTS = [
     (pins.test_adaptive_gnn_that_never_stops_is_the_fixed_depth_gnn, True),
     (pins.test_adaptive_gnn_stops_after_the_planted_layer, True),
     (pins.test_adaptive_decision_pools_the_points_of_the_batch, True),
+    (pins.test_pruning_mask_hand_built, False),
+    (pins.test_matchability_matches_torch_linear_sigmoid, False),
+    (pins.test_pruning_that_keeps_everything_is_the_unpruned_pass, True),
+    (pins.test_pruned_points_leave_the_later_layers, True),
+    (pins.test_pruned_points_are_unmatched_and_matches_map_back, True),
+    (pins.test_exit_share_counts_pruned_points_as_confident, True),
 ]
 
 
@@ -263,7 +269,8 @@ def _confidence_without_bias(x, w, b):
     return 1.0 / (1.0 + np.exp(-z))
 
 
-def _adaptive_last_pair_only(xs0, xs1, weights, heads, eps, depth_confidence, n_stages=None):
+def _adaptive_last_pair_only(xs0, xs1, weights, heads, eps, depth_confidence, n_stages=None,
+                             width_confidence=None, pruning_threshold=1536):
     stages = weights["stages"]
     n_stages = len(stages) if n_stages is None else n_stages
     n_layers = n_stages // 2
@@ -282,11 +289,60 @@ def _adaptive_last_pair_only(xs0, xs1, weights, heads, eps, depth_confidence, n_
         conf = O.token_confidence(np.concatenate([xs0[b], xs1[b]]), weights["tc_w"][layer],
                                   weights["tc_b"][layer])
         if O.check_if_stop(conf, layer, n_layers, depth_confidence, conf.size):
-            return xs0, xs1, layer + 1
-    return xs0, xs1, n_layers
+            return xs0, xs1, None, None, layer + 1
+    return xs0, xs1, None, None, n_layers
+
+
+def _mask_keeps_equal_score(confidences, scores, layer, n_layers, width_confidence):
+    keep = np.asarray(scores) >= (1.0 - width_confidence)
+    if confidences is not None:
+        keep = keep | (np.asarray(confidences) <= O.confidence_threshold(layer, n_layers))
+    return keep
+
+
+def _mask_prunes_uncertain(confidences, scores, layer, n_layers, width_confidence):
+    keep = np.asarray(scores) > (1.0 - width_confidence)
+    if confidences is not None:
+        keep = keep | (np.asarray(confidences) < O.confidence_threshold(layer, n_layers))
+    return keep
+
+
+_adaptive = O.attentional_gnn_adaptive
+
+
+def _adaptive_prunes_after_last_layer(xs0, xs1, weights, heads, eps, depth_confidence, n_stages=None,
+                                      width_confidence=None, pruning_threshold=1536):
+    xs0, xs1, kept0, kept1, layers = _adaptive(xs0, xs1, weights, heads, eps, depth_confidence, n_stages,
+                                               width_confidence, pruning_threshold)
+    if width_confidence is not None and width_confidence > 0:
+        last = layers - 1
+        n_layers = (len(weights["stages"]) if n_stages is None else n_stages) // 2
+        for b in range(len(xs0)):
+            for xs, kept in ((xs0, kept0), (xs1, kept1)):
+                if len(xs[b]) > pruning_threshold:
+                    s = O.matchability(xs[b], weights["mt_w"][last], weights["mt_b"][last])
+                    keep = O.get_pruning_mask(None, s, last, n_layers, width_confidence)
+                    xs[b], kept[b] = xs[b][keep], kept[b][keep]
+    return xs0, xs1, kept0, kept1, layers
+
+
+def _stop_over_points_left(confidences, layer, n_layers, depth_confidence, num_points):
+    c = np.asarray(confidences)
+    lam = O.confidence_threshold(layer, n_layers)
+    return 1.0 - float(np.sum(c < lam)) / float(c.size) > depth_confidence
+
+
+def _matchability_negated(x, w, b):
+    z = -(np.asarray(x, float) @ np.asarray(w, float) + float(b))
+    return 1.0 / (1.0 + np.exp(-z))
 
 
 MUTATIONS = {
+    "pruning keeps a score equal to 1 - width": ("get_pruning_mask", _mask_keeps_equal_score),
+    "uncertain points at the threshold pruned": ("get_pruning_mask", _mask_prunes_uncertain),
+    "pruning after the last layer": ("attentional_gnn_adaptive", _adaptive_prunes_after_last_layer),
+    "exit share over the points left": ("check_if_stop", _stop_over_points_left),
+    "matchability of the negated logit": ("matchability", _matchability_negated),
     "exit threshold grows with depth": ("confidence_threshold", _threshold_growing),
     "confidence at the threshold counted as low": ("check_if_stop", _stop_counts_equal_as_low),
     "exit when the share equals depth_confidence": ("check_if_stop", _stop_at_equal_share),

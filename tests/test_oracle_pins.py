@@ -503,7 +503,7 @@ def _adaptive_inputs(weights, B=2, M=9, N=7, seed=5):
 def test_adaptive_gnn_that_never_stops_is_the_fixed_depth_gnn(weights):
     xs0, xs1 = _adaptive_inputs(weights)
     # ratio > 1 is impossible: every layer runs
-    a0, a1, layers = O.attentional_gnn_adaptive(xs0, xs1, weights, 4, 1e-5, 1.0, n_stages=6)
+    a0, a1, _, _, layers = O.attentional_gnn_adaptive(xs0, xs1, weights, 4, 1e-5, 1.0, n_stages=6)
     assert layers == 3
     for b in range(2):
         r0, r1 = O.attentional_gnn(xs0[b], xs1[b], weights, 4, 1e-5, n_stages=6)
@@ -518,7 +518,7 @@ def test_adaptive_gnn_stops_after_the_planted_layer(weights):
     for k in (0, 1, 2):
         # classifiers certain "not confident" before layer k, "confident" at k
         w["tc_b"] = [-50.0 if l < k else 50.0 for l in range(9)]
-        a0, a1, layers = O.attentional_gnn_adaptive(xs0, xs1, w, 4, 1e-5, 0.95, n_stages=8)
+        a0, a1, _, _, layers = O.attentional_gnn_adaptive(xs0, xs1, w, 4, 1e-5, 0.95, n_stages=8)
         assert layers == k + 1
         for b in range(2):
             r0, r1 = O.attentional_gnn(xs0[b], xs1[b], w, 4, 1e-5, n_stages=2 * k + 2)
@@ -526,7 +526,7 @@ def test_adaptive_gnn_stops_after_the_planted_layer(weights):
             np.testing.assert_allclose(a1[b], r1, rtol=0, atol=1e-12)
     # no exit check after the last layer: a confident last layer changes nothing
     w["tc_b"] = [-50.0, -50.0, -50.0, 50.0] + [50.0] * 5
-    assert O.attentional_gnn_adaptive(xs0, xs1, w, 4, 1e-5, 0.95, n_stages=8)[2] == 4
+    assert O.attentional_gnn_adaptive(xs0, xs1, w, 4, 1e-5, 0.95, n_stages=8)[4] == 4
 
 
 def test_adaptive_decision_pools_the_points_of_the_batch(weights):
@@ -543,9 +543,151 @@ def test_adaptive_decision_pools_the_points_of_the_batch(weights):
     xs1 = [np.abs(xs1[0]) + 50.0, -np.abs(xs1[1]) - 50.0]
     # one stage pair changes the states, so look at the layer-0 confidences
     # after the first layer, as the gnn does
-    a0, a1, _ = O.attentional_gnn_adaptive(xs0, xs1, w, 4, 1e-5, 1.0, n_stages=2)
+    a0, a1, _, _, _ = O.attentional_gnn_adaptive(xs0, xs1, w, 4, 1e-5, 1.0, n_stages=2)
     conf = np.concatenate([O.token_confidence(np.concatenate([a0[b], a1[b]]), tw, 0.0) for b in range(2)])
     share = 1.0 - np.mean(conf < O.confidence_threshold(0, 2))
     assert 0.0 < share < 1.0
-    assert O.attentional_gnn_adaptive(xs0, xs1, w, 4, 1e-5, share - 1e-9, n_stages=4)[2] == 1
-    assert O.attentional_gnn_adaptive(xs0, xs1, w, 4, 1e-5, share, n_stages=4)[2] == 2
+    assert O.attentional_gnn_adaptive(xs0, xs1, w, 4, 1e-5, share - 1e-9, n_stages=4)[4] == 1
+    assert O.attentional_gnn_adaptive(xs0, xs1, w, 4, 1e-5, share, n_stages=4)[4] == 2
+
+
+# --------------------------------------------------------------------------- point pruning
+def test_pruning_mask_hand_built():
+    lam = O.confidence_threshold(1, 9)
+    scores = np.array([0.5, 0.01, 0.001, 0.001, 0.001, 0.0100001])
+    conf = np.array([0.99, 0.99, lam, lam + 1e-9, 0.2, 0.99])
+    # score above 1 - 0.99 keeps; a confidence not above lambda keeps (never pruned)
+    keep = O.get_pruning_mask(conf, scores, 1, 9, 0.99)
+    assert keep.tolist() == [True, False, True, False, True, True]
+    # without confidences (the exit disabled) only the score decides
+    assert O.get_pruning_mask(None, scores, 1, 9, 0.99).tolist() == [True, False, False, False, False, True]
+    # strictly above 1 - width_confidence (0.5 is exact in binary)
+    assert O.get_pruning_mask(None, np.array([0.5, 0.5000001]), 1, 9, 0.5).tolist() == [False, True]
+
+
+def test_matchability_matches_torch_linear_sigmoid():
+    rng = np.random.default_rng(43)
+    x = rng.standard_normal((21, 256))
+    w = rng.standard_normal(256) * 0.2
+    lin = torch.nn.Linear(256, 1).double()
+    with torch.no_grad():
+        lin.weight.copy_(torch.from_numpy(w)[None])
+        lin.bias.fill_(-0.3)
+        ref = torch.sigmoid(lin(torch.from_numpy(x)))[:, 0].numpy()
+    np.testing.assert_allclose(O.matchability(x, w, -0.3), ref, rtol=0, atol=1e-15)
+
+
+def _pruning_weights(weights, n_layers=9):
+    # matchability sigmoid(1e4 x[0]): about 1 where channel 0 of the state is
+    # positive and about 0 where it is negative (beyond 5e-4 either way)
+    w = dict(weights)
+    mw = np.zeros(256)
+    mw[0] = 1e4
+    w["mt_w"] = [mw] * n_layers
+    w["mt_b"] = [0.0] * n_layers
+    return w
+
+
+def test_pruning_that_keeps_everything_is_the_unpruned_pass(weights):
+    xs0, xs1 = _adaptive_inputs(weights, B=2, M=9, N=7)
+    w = weights                                  # generated matchability: every score is above 0
+    a = O.attentional_gnn_adaptive(xs0, xs1, w, 4, 1e-5, None, 6, width_confidence=1.0, pruning_threshold=0)
+    r = O.attentional_gnn_adaptive(xs0, xs1, w, 4, 1e-5, None, 6)
+    for b in range(2):
+        np.testing.assert_array_equal(a[2][b], np.arange(9))
+        np.testing.assert_allclose(a[0][b], r[0][b], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(a[1][b], r[1][b], rtol=0, atol=1e-12)
+    # an image with no more points than the threshold is never pruned
+    w = _pruning_weights(weights)
+    a = O.attentional_gnn_adaptive(xs0, xs1, w, 4, 1e-5, None, 6, width_confidence=0.99, pruning_threshold=9)
+    assert all(len(k) == 9 for k in a[2]) and all(len(k) == 7 for k in a[3])
+
+
+def _pruned_reference(xs0, xs1, w, keep_channel_positive=True):
+    """Layer 0 on every point, then layer 1 on the points whose channel 0 is
+    positive after layer 0: the pruned two-layer pass written as a composition
+    of the fixed-depth GNN."""
+    refs = []
+    stages_rest = dict(w)
+    stages_rest["stages"] = w["stages"][2:]
+    for x0, x1 in zip(xs0, xs1):
+        y0, y1 = O.attentional_gnn(x0, x1, w, 4, 1e-5, n_stages=2)
+        k0, k1 = np.where(y0[:, 0] > 0)[0], np.where(y1[:, 0] > 0)[0]
+        margin = min(np.abs(y0[:, 0]).min(), np.abs(y1[:, 0]).min())
+        z0, z1 = O.attentional_gnn(y0[k0], y1[k1], stages_rest, 4, 1e-5, n_stages=2)
+        refs.append((z0, z1, k0, k1, margin))
+    return refs
+
+
+def test_pruned_points_leave_the_later_layers(weights):
+    xs0, xs1 = _adaptive_inputs(weights, B=2, M=12, N=10, seed=8)
+    w = _pruning_weights(weights)
+    # two layers: pruning after layer 0 only (never after the last layer)
+    a0, a1, k0, k1, layers = O.attentional_gnn_adaptive(xs0, xs1, w, 4, 1e-5, None, 4,
+                                                          width_confidence=0.99, pruning_threshold=0)
+    assert layers == 2
+    for b, (z0, z1, r0, r1, margin) in enumerate(_pruned_reference(xs0, xs1, w)):
+        assert margin > 2e-3                     # sigmoid(1e4 x) is decidable on both sides
+        assert 0 < len(r0) < 12 and 0 < len(r1) < 10
+        np.testing.assert_array_equal(k0[b], r0)
+        np.testing.assert_array_equal(k1[b], r1)
+        np.testing.assert_allclose(a0[b], z0, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(a1[b], z1, rtol=0, atol=1e-12)
+
+
+def test_pruned_points_are_unmatched_and_matches_map_back(weights):
+    rng = np.random.default_rng(21)
+    pairs = [synth.make_pair(rng, 12, 10, 0.6) for _ in range(2)]
+    batch = {k: np.stack([p[k] for p in pairs]) for k in ("kpts0", "conf0", "desc0", "kpts1", "conf1", "desc1")}
+    w = _pruning_weights(weights)
+    out, layers = O.superglue_batch_adaptive(batch, w, None, n_stages=4, width_confidence=0.99,
+                                             pruning_threshold=0)
+    for b, res in enumerate(out):
+        k0, k1 = res["kept0"], res["kept1"]
+        gone0 = np.setdiff1d(np.arange(12), k0)
+        gone1 = np.setdiff1d(np.arange(10), k1)
+        assert np.all(res["matches0"][gone0] == -1) and np.all(res["mscores0"][gone0] == 0)
+        assert np.all(res["matches1"][gone1] == -1) and np.all(res["mscores1"][gone1] == 0)
+        assert res["log_P"].shape == (len(k0) + 1, len(k1) + 1)
+        # the head on the points left, in their own indices, agrees after the map
+        sub = O.extract_matches(res["log_P"], 0.2)
+        for p, i in enumerate(k0):
+            j = res["matches0"][i]
+            assert (j == -1) == (sub[0][p] == -1)
+            if j >= 0:
+                assert j == k1[sub[0][p]] and res["matches1"][j] == i
+
+
+def test_exit_share_counts_pruned_points_as_confident(weights):
+    # layer 0: confident where channel 1 is positive (about half), matchability
+    # 0 everywhere, so exactly the confident points are pruned and the share at
+    # layer 0 stays below depth_confidence; layer 1: confident where channel 2
+    # is positive.  With the original point count a pruned point counts as
+    # confident, which puts the share at layer 1 above the one of the points
+    # left alone
+    xs0, xs1 = _adaptive_inputs(weights, B=1, M=16, N=14, seed=12)
+    w = dict(weights)
+    w["mt_w"] = [np.zeros(256)] * 9
+    w["mt_b"] = [-50.0] * 9
+    t0, t1 = np.zeros(256), np.zeros(256)
+    t0[1], t1[2] = 100.0, 100.0
+    w["tc_w"] = [t0, t1] + [np.zeros(256)] * 7
+    w["tc_b"] = [0.0] * 9
+    total = 30
+    a0, a1, k0, k1, _ = O.attentional_gnn_adaptive(xs0, xs1, w, 4, 1e-5, 1.0, 4, width_confidence=0.99,
+                                                   pruning_threshold=0)
+    left = len(k0[0]) + len(k1[0])
+    assert 0 < left < total
+    # confidences of the points left after layer 1 (the run above never exits)
+    y0, y1, _, _, _ = O.attentional_gnn_adaptive(xs0, xs1, w, 4, 1e-5, 1.0, 6, width_confidence=0.99,
+                                                 pruning_threshold=0)
+    c = O.token_confidence(np.concatenate([y0[0], y1[0]]), t1, 0.0)
+    low = int(np.sum(c < O.confidence_threshold(1, 3)))
+    share_all, share_left = 1.0 - low / total, 1.0 - low / left
+    share0 = 1.0 - (total - (total - left)) / total     # layer 0: the pruned points were the confident ones
+    assert share0 < share_all
+    d = (max(share0, share_left) + share_all) / 2.0 if share_left < share_all else None
+    if d is None or not (share0 < d < share_all):
+        pytest.skip(f"no separating depth_confidence: {share0}, {share_left}, {share_all}")
+    assert O.attentional_gnn_adaptive(xs0, xs1, w, 4, 1e-5, d, 6, width_confidence=0.99,
+                                      pruning_threshold=0)[4] == 2
