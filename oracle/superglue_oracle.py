@@ -139,6 +139,31 @@ def multi_head_attention(x, src, st, heads):
     return linear(msg, st["Wm"], st["bm"])
 
 
+def bidirectional_cross_attention(x0, x1, st, heads):
+    """Cross attention with one similarity matrix for both directions [LightGlue
+    review, section 2.3 交叉注意力, the CrossBlock forward listing]: a point has
+    one projection qk = Wqk x + bqk (here st["Wq"], st["bq"]) and a value
+    v = Wv x + bv; per head, sim = (qk0 s)(qk1 s)^T with s = d_head^(-1/4);
+    softmax over the rows of sim gives the messages to image 0 from the values
+    of image 1, softmax over the rows of sim^T the messages to image 1; the
+    concatenated heads go through the merge layer.  Returns (m0, m1)."""
+    qk0 = linear(x0, st["Wq"], st["bq"])
+    qk1 = linear(x1, st["Wq"], st["bq"])
+    v0 = linear(x0, st["Wv"], st["bv"])
+    v1 = linear(x1, st["Wv"], st["bv"])
+    d = qk0.shape[1]
+    dh = d // heads
+    s = dh ** -0.25
+    m0 = np.empty((x0.shape[0], d), F64)
+    m1 = np.empty((x1.shape[0], d), F64)
+    for h in range(heads):
+        sl = slice(h * dh, (h + 1) * dh)
+        sim = (qk0[:, sl] * s) @ (qk1[:, sl] * s).T
+        m0[:, sl] = softmax(sim, axis=1) @ v1[:, sl]
+        m1[:, sl] = softmax(sim.T, axis=1) @ v0[:, sl]
+    return linear(m0, st["Wm"], st["bm"]), linear(m1, st["Wm"], st["bm"])
+
+
 def attentional_propagation(x, src, st, heads, eps):
     """delta = MLP([x || message]), MLP 512-512-256 with BN+ReLU in the middle
     and last bias 0 [realcat notes, section 多层GNN, AttentionalPropagation]."""

@@ -48,6 +48,8 @@ PIN_TESTS = [
     (pins.test_pruned_points_leave_the_later_layers, True),
     (pins.test_pruned_points_are_unmatched_and_matches_map_back, True),
     (pins.test_exit_share_counts_pruned_points_as_confident, True),
+    (pins.test_bidirectional_cross_attention_is_tied_cross_attention_in_torch, True),
+    (pins.test_bidirectional_cross_attention_on_one_point_each, False),
 ]
 
 
@@ -337,7 +339,27 @@ def _matchability_negated(x, w, b):
     return 1.0 / (1.0 + np.exp(-z))
 
 
+def _bidir_same_softmax_axis(x0, x1, st, heads):
+    qk0 = O.linear(x0, st["Wq"], st["bq"])
+    qk1 = O.linear(x1, st["Wq"], st["bq"])
+    v0 = O.linear(x0, st["Wv"], st["bv"])
+    v1 = O.linear(x1, st["Wv"], st["bv"])
+    d = qk0.shape[1]
+    dh = d // heads
+    s = dh ** -0.25
+    m0 = np.empty((x0.shape[0], d))
+    m1 = np.empty((x1.shape[0], d))
+    for h in range(heads):
+        sl = slice(h * dh, (h + 1) * dh)
+        sim = (qk0[:, sl] * s) @ (qk1[:, sl] * s).T
+        a = O.softmax(sim, axis=1)
+        m0[:, sl] = a @ v1[:, sl]
+        m1[:, sl] = a.T @ v0[:, sl]             # the row softmax reused for the other direction
+    return O.linear(m0, st["Wm"], st["bm"]), O.linear(m1, st["Wm"], st["bm"])
+
+
 MUTATIONS = {
+    "bidirectional: one softmax axis for both directions": ("bidirectional_cross_attention", _bidir_same_softmax_axis),
     "pruning keeps a score equal to 1 - width": ("get_pruning_mask", _mask_keeps_equal_score),
     "uncertain points at the threshold pruned": ("get_pruning_mask", _mask_prunes_uncertain),
     "pruning after the last layer": ("attentional_gnn_adaptive", _adaptive_prunes_after_last_layer),

@@ -691,3 +691,33 @@ def test_exit_share_counts_pruned_points_as_confident(weights):
         pytest.skip(f"no separating depth_confidence: {share0}, {share_left}, {share_all}")
     assert O.attentional_gnn_adaptive(xs0, xs1, w, 4, 1e-5, d, 6, width_confidence=0.99,
                                       pruning_threshold=0)[4] == 2
+
+
+# --------------------------------------------------------------------------- bidirectional cross attention
+def test_bidirectional_cross_attention_is_tied_cross_attention_in_torch(weights):
+    # with one projection for queries and keys, the two directions of torch's
+    # MultiheadAttention are the row softmax of sim and the row softmax of sim^T
+    rng = np.random.default_rng(44)
+    x0 = rng.standard_normal((13, 256)) * 0.3
+    x1 = rng.standard_normal((9, 256)) * 0.3
+    st = dict(weights["stages"][1])
+    st["Wk"], st["bk"] = st["Wq"], st["bq"]
+    mha = _torch_mha(st)
+    with torch.no_grad():
+        r0, _ = mha(torch.tensor(x0[None]), torch.tensor(x1[None]), torch.tensor(x1[None]))
+        r1, _ = mha(torch.tensor(x1[None]), torch.tensor(x0[None]), torch.tensor(x0[None]))
+    m0, m1 = O.bidirectional_cross_attention(x0, x1, st, 4)
+    np.testing.assert_allclose(m0, r0[0].numpy(), rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(m1, r1[0].numpy(), rtol=1e-11, atol=1e-12)
+
+
+def test_bidirectional_cross_attention_on_one_point_each():
+    # one point per image: every softmax is over a single entry, so each
+    # message is the other point's value through the merge layer
+    rng = np.random.default_rng(45)
+    st = {k: rng.standard_normal((8, 8)) for k in ("Wq", "Wv", "Wm")}
+    st.update({k: rng.standard_normal(8) for k in ("bq", "bv", "bm")})
+    x0, x1 = rng.standard_normal((1, 8)), rng.standard_normal((1, 8))
+    m0, m1 = O.bidirectional_cross_attention(x0, x1, st, 2)
+    np.testing.assert_allclose(m0[0], (st["Wv"] @ x1[0] + st["bv"]) @ st["Wm"].T + st["bm"], rtol=1e-12)
+    np.testing.assert_allclose(m1[0], (st["Wv"] @ x0[0] + st["bv"]) @ st["Wm"].T + st["bm"], rtol=1e-12)
