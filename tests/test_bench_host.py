@@ -48,3 +48,19 @@ def test_algorithmic_work_matches_the_pages_counts():
     bound, bytes_ = w["sinkhorn"]
     assert bound == "hbm"
     assert bytes_ == 2 * 100 * 4 * 2049 * 2049
+
+
+def test_planted_exit_weights_make_the_oracle_exit_after_the_layer():
+    # the classifiers bench.py plants for --exit-layer K: the oracle's adaptive
+    # GNN stops after layer K (its confidences are 0 before K and 1 at K)
+    import numpy as np
+    from learned_sparse_feature_b200 import synth
+    from oracle import superglue_oracle as O
+    w = bench.planted_exit_weights(synth.make_weights(0), 1)
+    rng = np.random.default_rng(3)
+    xs0 = [rng.standard_normal((5, 256))]
+    xs1 = [rng.standard_normal((4, 256))]
+    assert O.attentional_gnn_adaptive(xs0, xs1, w, 4, 1e-5, bench.EXIT_DEPTH_CONFIDENCE, 6)[4] == 2
+    c = bench._config(synth.WORKLOADS["pair2048"], 1, "sinkhorn", 1)
+    assert c["adaptive_depth"]["exit_after_layer"] == 1
+    assert "adaptive_depth" not in bench._config(synth.WORKLOADS["pair2048"], 1)
