@@ -327,6 +327,81 @@ def double_softmax_head(x0, x1, Wp, bp, wz, bz):
     return double_softmax_log_assignment(sim, z0, z1), sim, z0, z1
 
 
+# --------------------------------------------------------------------------- training-side derivatives
+def nll_loss(logP, matches, unmatched0, unmatched1):
+    """Negative log-likelihood of the augmented assignment: -sum log P_ij over the
+    true matches, -sum log P_i,N+1 over the unmatched points of A, -sum
+    log P_M+1,j over those of B [realcat notes, section Loss]."""
+    logP = _as64(logP)
+    M, N = logP.shape[0] - 1, logP.shape[1] - 1
+    loss = -sum(logP[i, j] for i, j in matches)
+    loss -= sum(logP[i, N] for i in unmatched0)
+    loss -= sum(logP[M, j] for j in unmatched1)
+    return float(loss)
+
+
+def nll_loss_grad(shape, matches, unmatched0, unmatched1):
+    """d nll_loss / d log P: -1 at every entry the loss reads."""
+    g = np.zeros(shape, F64)
+    M, N = shape[0] - 1, shape[1] - 1
+    for i, j in matches:
+        g[i, j] -= 1.0
+    for i in unmatched0:
+        g[i, N] -= 1.0
+    for j in unmatched1:
+        g[M, j] -= 1.0
+    return g
+
+
+def attend_backward(q, k, v, g):
+    """Gradients of m = softmax(q k^T / sqrt(d)) v for the upstream gradient g =
+    dL/dm: dL/de_ij = alpha_ij g_i . (v_j - m_i) for the scores e [huluoboge
+    blog, the derivation of how the loss changes attention], then through
+    e = q k^T / sqrt(d) and m = alpha v.  Returns (dq, dk, dv)."""
+    q, k, v, g = _as64(q), _as64(k), _as64(v), _as64(g)
+    d = q.shape[1]
+    m, a = attend(q, k, v)
+    de = a * (g @ v.T - np.sum(g * m, axis=1, keepdims=True))
+    dq = de @ k / math.sqrt(d)
+    dk = de.T @ q / math.sqrt(d)
+    dv = a.T @ g
+    return dq, dk, dv
+
+
+def log_sinkhorn_backward(Z, log_mu, log_nu, iters, G):
+    """dL/dZ for out = log_sinkhorn(Z, ...) and the upstream gradient G = dL/dout,
+    by reverse mode through the T iterations: out = Z + u_T + v_T; v_t = log nu -
+    LSE_i(Z + u_t) gives dv_t/dZ_ij = dv_t/du_t,i = -Pc_ij (Pc the softmax of Z + u_t
+    over i); u_t = log mu - LSE_j(Z + v_{t-1}) gives -Pr_ij (Pr the softmax of
+    Z + v_{t-1} over j); v_0 = 0."""
+    Z, G = _as64(Z), _as64(G)
+    us, vs = [], [np.zeros(Z.shape[1], F64)]
+    u = np.zeros(Z.shape[0], F64)
+    v = vs[0]
+    for _ in range(iters):
+        u = log_mu - logsumexp(Z + v[None, :], axis=1)
+        v = log_nu - logsumexp(Z + u[:, None], axis=0)
+        us.append(u)
+        vs.append(v)
+    dZ = G.copy()
+    if iters == 0:
+        return dZ
+    gu = G.sum(axis=1)
+    gv = G.sum(axis=0)
+    for t in range(iters, 0, -1):
+        u_t, v_prev = us[t - 1], vs[t - 1]
+        x = Z + u_t[:, None]
+        pc = np.exp(x - logsumexp(x, axis=0)[None, :])          # columns sum to 1
+        dZ -= pc * gv[None, :]
+        gu = gu - (pc * gv[None, :]).sum(axis=1)
+        y = Z + v_prev[None, :]
+        pr = np.exp(y - logsumexp(y, axis=1)[:, None])          # rows sum to 1
+        dZ -= pr * gu[:, None]
+        gv = -(pr * gu[:, None]).sum(axis=0)
+        gu = np.zeros_like(gu)
+    return dZ
+
+
 # --------------------------------------------------------------------------- adaptive depth
 def confidence_threshold(layer, n_layers):
     """Per-layer exit threshold lambda_l = clip(0.8 + 0.1 exp(-4 l / L), 0, 1)

@@ -50,6 +50,10 @@ PIN_TESTS = [
     (pins.test_exit_share_counts_pruned_points_as_confident, True),
     (pins.test_bidirectional_cross_attention_is_tied_cross_attention_in_torch, True),
     (pins.test_bidirectional_cross_attention_on_one_point_each, False),
+    (pins.test_nll_loss_hand_built, False),
+    (pins.test_attend_backward_matches_autograd, False),
+    (pins.test_log_sinkhorn_backward_matches_autograd, False),
+    (pins.test_log_sinkhorn_backward_by_finite_differences, False),
 ]
 
 
@@ -358,7 +362,29 @@ def _bidir_same_softmax_axis(x0, x1, st, heads):
     return O.linear(m0, st["Wm"], st["bm"]), O.linear(m1, st["Wm"], st["bm"])
 
 
+def _nll_matches_only(logP, matches, unmatched0, unmatched1):
+    logP = np.asarray(logP, float)
+    return float(-sum(logP[i, j] for i, j in matches))
+
+
+def _attend_backward_no_mean(q, k, v, g):
+    d = q.shape[1]
+    m, a = O.attend(q, k, v)
+    de = a * (g @ v.T)
+    return de @ k / math.sqrt(d), de.T @ q / math.sqrt(d), a.T @ g
+
+
+_sk_bwd = O.log_sinkhorn_backward
+
+
+def _sinkhorn_backward_last_iteration_only(Z, log_mu, log_nu, iters, G):
+    return _sk_bwd(Z, log_mu, log_nu, min(iters, 1), G)
+
+
 MUTATIONS = {
+    "NLL loss without the unmatched terms": ("nll_loss", _nll_matches_only),
+    "attention gradient without the mean message": ("attend_backward", _attend_backward_no_mean),
+    "Sinkhorn gradient through one iteration": ("log_sinkhorn_backward", _sinkhorn_backward_last_iteration_only),
     "bidirectional: one softmax axis for both directions": ("bidirectional_cross_attention", _bidir_same_softmax_axis),
     "pruning keeps a score equal to 1 - width": ("get_pruning_mask", _mask_keeps_equal_score),
     "uncertain points at the threshold pruned": ("get_pruning_mask", _mask_prunes_uncertain),

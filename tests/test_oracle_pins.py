@@ -721,3 +721,75 @@ def test_bidirectional_cross_attention_on_one_point_each():
     m0, m1 = O.bidirectional_cross_attention(x0, x1, st, 2)
     np.testing.assert_allclose(m0[0], (st["Wv"] @ x1[0] + st["bv"]) @ st["Wm"].T + st["bm"], rtol=1e-12)
     np.testing.assert_allclose(m1[0], (st["Wv"] @ x0[0] + st["bv"]) @ st["Wm"].T + st["bm"], rtol=1e-12)
+
+
+# --------------------------------------------------------------------------- training-side derivatives
+def test_nll_loss_hand_built():
+    logP = np.log(np.array([[0.5, 0.2, 0.3], [0.1, 0.6, 0.3], [0.4, 0.2, 1.4]]))
+    loss = O.nll_loss(logP, [(0, 0)], [1], [1])
+    assert loss == pytest.approx(-(math.log(0.5) + math.log(0.3) + math.log(0.2)), abs=1e-15)
+    g = O.nll_loss_grad(logP.shape, [(0, 0)], [1], [1])
+    assert g[0, 0] == -1 and g[1, 2] == -1 and g[2, 1] == -1 and np.count_nonzero(g) == 3
+
+
+def test_attend_backward_matches_autograd():
+    rng = np.random.default_rng(46)
+    q, k, v = rng.standard_normal((7, 16)), rng.standard_normal((9, 16)), rng.standard_normal((9, 16))
+    g = rng.standard_normal((7, 16))
+    tq, tk, tv = (torch.tensor(a, requires_grad=True) for a in (q, k, v))
+    a = torch.softmax(tq @ tk.T / 4.0, dim=1)
+    (a @ tv).backward(torch.tensor(g))
+    dq, dk, dv = O.attend_backward(q, k, v, g)
+    np.testing.assert_allclose(dq, tq.grad.numpy(), rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(dk, tk.grad.numpy(), rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(dv, tv.grad.numpy(), rtol=1e-12, atol=1e-13)
+
+
+def test_attention_score_gradient_formula_of_the_pages():
+    # dL/de_ij = alpha_ij g_i . (v_j - m_i): autograd through softmax(e) v
+    rng = np.random.default_rng(47)
+    e, v, g = rng.standard_normal((5, 6)), rng.standard_normal((6, 3)), rng.standard_normal((5, 3))
+    te = torch.tensor(e, requires_grad=True)
+    (torch.softmax(te, 1) @ torch.tensor(v)).backward(torch.tensor(g))
+    a = np.exp(e - e.max(1, keepdims=True))
+    a /= a.sum(1, keepdims=True)
+    m = a @ v
+    formula = np.array([[a[i, j] * g[i] @ (v[j] - m[i]) for j in range(6)] for i in range(5)])
+    np.testing.assert_allclose(te.grad.numpy(), formula, rtol=1e-12, atol=1e-14)
+
+
+def test_log_sinkhorn_backward_matches_autograd():
+    rng = np.random.default_rng(48)
+    S = rng.standard_normal((4, 5)) * 2.0
+    Z = O.augment_dustbin(S, 0.7)
+    log_mu, log_nu, _ = O.log_marginals(4, 5)
+    G = rng.standard_normal(Z.shape)
+    tz = torch.tensor(Z, requires_grad=True)
+    tmu, tnu = torch.tensor(log_mu), torch.tensor(log_nu)
+    u = torch.zeros(5, dtype=torch.float64)
+    v = torch.zeros(6, dtype=torch.float64)
+    for _ in range(7):
+        u = tmu - torch.logsumexp(tz + v[None, :], dim=1)
+        v = tnu - torch.logsumexp(tz + u[:, None], dim=0)
+    (tz + u[:, None] + v[None, :]).backward(torch.tensor(G))
+    np.testing.assert_allclose(O.log_sinkhorn_backward(Z, log_mu, log_nu, 7, G), tz.grad.numpy(),
+                               rtol=1e-11, atol=1e-12)
+    # no iterations: the identity
+    np.testing.assert_allclose(O.log_sinkhorn_backward(Z, log_mu, log_nu, 0, G), G, rtol=0, atol=0)
+
+
+def test_log_sinkhorn_backward_by_finite_differences():
+    # the NLL loss of a planted match through 20 iterations, central differences
+    rng = np.random.default_rng(49)
+    Z = O.augment_dustbin(rng.standard_normal((3, 3)), 1.0)
+    log_mu, log_nu, _ = O.log_marginals(3, 3)
+    matches, un0, un1 = [(0, 1), (2, 0)], [1], [2]
+    loss = lambda z: O.nll_loss(O.log_sinkhorn(z, log_mu, log_nu, 20), matches, un0, un1)
+    G = O.nll_loss_grad(Z.shape, matches, un0, un1)
+    grad = O.log_sinkhorn_backward(Z, log_mu, log_nu, 20, G)
+    h = 1e-6
+    for i, j in [(0, 0), (0, 1), (1, 3), (3, 2), (2, 0)]:
+        zp, zm = Z.copy(), Z.copy()
+        zp[i, j] += h
+        zm[i, j] -= h
+        assert abs((loss(zp) - loss(zm)) / (2 * h) - grad[i, j]) < 1e-6
