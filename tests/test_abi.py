@@ -60,3 +60,27 @@ def test_create_rejects_bad_arguments(lib):
     cfg = binding.SgConfig(256, 4, 18, 100, 0.2, 1e-5, 5, 640.0, 480.0, 0, 1, 64, 64)
     assert lib.sg_create(C.byref(w), C.byref(cfg), C.byref(h)) == 1     # bad precision
     assert not h.value
+
+
+def test_header_is_plain_c_and_links_against_the_library(lib, tmp_path):
+    # a C99 translation unit that includes the header and takes the address of
+    # every declared entry point, linked against the built library: the boundary
+    # needs no C++ and no torch
+    from learned_sparse_feature_b200 import binding
+    names = _declared()
+    src = tmp_path / "abi_check.c"
+    body = "\n".join(f"    (void (*)(void)){n}," for n in names)
+    src.write_text(f'#include "sg.h"\n#include <stdio.h>\n'
+                   f"void (*entry_points[])(void) = {{\n{body}\n}};\n"
+                   "int main(void) {\n"
+                   "    sg_weights w = {0};\n    sg_config c = {0};\n    sg_handle *h = 0;\n"
+                   "    (void)w; (void)c; (void)h;\n"
+                   '    printf("%d\\n", (int)(sizeof entry_points / sizeof entry_points[0]));\n'
+                   "    return 0;\n}\n")
+    exe = tmp_path / "abi_check"
+    libdir = os.path.dirname(binding.LIB_PATH)
+    r = subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic",
+                        "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe),
+                        "-L", libdir, "-lsg", f"-Wl,-rpath,{libdir}", "-Wl,--unresolved-symbols=ignore-in-shared-libs"],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
