@@ -227,7 +227,8 @@ sg_status_t sg_status(sg_handle* h, void* stream);
 /*
  * Adaptive depth: synchronises `stream` and writes to *layers how many
  * (self, cross) layers the last sg_match / sg_scores on this handle ran
- * (ceil(n_stages / 2) when adaptive depth is off or no exit was taken).
+ * (ceil(n_stages / 2) when adaptive depth is off or no exit was taken; 0 after
+ * a call with M == 0 or N == 0).
  * The skipped layers' kernels still launch and return at once; the final
  * projection and the matching head run on the states at the exit.
  * Returns SG_ERR_INVALID_ARG for a null pointer, SG_ERR_CUDA if the stream

@@ -70,6 +70,7 @@ struct sg_handle {
   // adaptive depth (cfg.depth_confidence > 0): per-layer token-confidence
   // classifiers and the pass's stop / count words
   bool adaptive;
+  bool last_empty;     // the last sg_match had no points on one side: no layer ran
   float* tc_w[SG_MAX_STAGES / 2];
   float tc_b[SG_MAX_STAGES / 2];
   unsigned* depth_words;
@@ -653,6 +654,7 @@ sg_status_t sg_scores(sg_handle* h, int B, int M, int N, const float* kpts0, con
   if (M == 0 || N == 0) return SG_ERR_SHAPE;
   if (!kpts0 || !conf0 || !desc0 || !kpts1 || !conf1 || !desc1 || !out_scores)
     return SG_ERR_INVALID_ARG;
+  h->last_empty = false;
   cudaStream_t s = (cudaStream_t)stream;
   Inputs in{kpts0, conf0, desc0, kpts1, conf1, desc1};
   int launches = 0;
@@ -704,6 +706,7 @@ sg_status_t sg_match(sg_handle* h, int B, int M, int N, const float* kpts0, cons
   if (st != SG_OK) return st;
   cudaStream_t s = (cudaStream_t)stream;
   if (B == 0) return SG_OK;
+  h->last_empty = (M == 0 || N == 0);
   if (M == 0 || N == 0) return empty_outputs(h, B, M, N, matches0, matches1, mscores0, mscores1, s);
   if (!kpts0 || !conf0 || !desc0 || !kpts1 || !conf1 || !desc1 || !matches0 || !matches1 ||
       !mscores0 || !mscores1)
@@ -834,6 +837,10 @@ int sg_profile_read(sg_handle* h, float* ms_by_class, int* launches_by_class, in
 sg_status_t sg_layers_run(sg_handle* h, int* layers, void* stream) {
   if (!h || !layers) return SG_ERR_INVALID_ARG;
   const int all = (h->cfg.n_stages + 1) / 2;
+  if (h->last_empty) {                 // M == 0 or N == 0: the early return ran no layer
+    *layers = 0;
+    return SG_OK;
+  }
   if (!h->adaptive) {
     *layers = all;
     return SG_OK;

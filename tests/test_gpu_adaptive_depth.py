@@ -145,3 +145,19 @@ def test_odd_stage_count_is_refused(dev, weights):
     from learned_sparse_feature_b200.binding import Matcher, SgError
     with pytest.raises(SgError):
         Matcher(weights, 1, 16, 16, n_stages=7, depth_confidence=0.95)
+
+
+def test_layers_run_after_an_empty_call_is_zero(dev, weights):
+    from learned_sparse_feature_b200.binding import Matcher
+    w = _planted(weights, 1)
+    m = Matcher(w, 1, 16, 16, n_stages=STAGES, depth_confidence=0.95)
+    k0, c0, d0 = torch.zeros((1, 0, 2), device=dev), torch.zeros((1, 0), device=dev), torch.zeros((1, 0, 256), device=dev)
+    k1, c1, d1 = torch.zeros((1, 5, 2), device=dev), torch.zeros((1, 5), device=dev), torch.zeros((1, 5, 256), device=dev)
+    m0 = torch.empty((1, 0), dtype=torch.int32, device=dev)
+    m1 = torch.empty((1, 5), dtype=torch.int32, device=dev)
+    s0, s1 = torch.empty((1, 0), device=dev), torch.empty((1, 5), device=dev)
+    m.match(k0, c0, d0, k1, c1, d1, None, m0, m1, s0, s1)
+    assert m.status() == 0
+    assert m.layers_run() == 0
+    assert (m1 == -1).all()
+    m.close()
