@@ -84,3 +84,26 @@ def test_header_is_plain_c_and_links_against_the_library(lib, tmp_path):
                         "-L", libdir, "-lsg", f"-Wl,-rpath,{libdir}", "-Wl,--unresolved-symbols=ignore-in-shared-libs"],
                        capture_output=True, text=True)
     assert r.returncode == 0, r.stderr
+
+
+def test_binding_structs_match_the_header_layout(tmp_path):
+    # the ctypes mirrors of sg_weights / sg_config must have the C layout: a C
+    # program prints sizeof and offsetof of every field, compared field by field
+    from learned_sparse_feature_b200 import binding
+    lines = []
+    for cname, cls in (("sg_weights", binding.SgWeights), ("sg_config", binding.SgConfig)):
+        lines.append(f'    printf("{cname} %zu\\n", sizeof({cname}));')
+        for f, _ in cls._fields_:
+            lines.append(f'    printf("{cname}.{f} %zu\\n", offsetof({cname}, {f}));')
+    src = tmp_path / "layout.c"
+    src.write_text('#include <stddef.h>\n#include <stdio.h>\n#include "sg.h"\nint main(void) {\n'
+                   + "\n".join(lines) + "\n    return 0;\n}\n")
+    exe = tmp_path / "layout"
+    r = subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                        str(src), "-o", str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    got = dict(l.split() for l in subprocess.run([str(exe)], capture_output=True, text=True).stdout.split("\n") if l)
+    for cname, cls in (("sg_weights", binding.SgWeights), ("sg_config", binding.SgConfig)):
+        assert int(got[cname]) == C.sizeof(cls), cname
+        for f, _ in cls._fields_:
+            assert int(got[f"{cname}.{f}"]) == getattr(cls, f).offset, f"{cname}.{f}"
