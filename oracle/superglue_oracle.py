@@ -177,14 +177,24 @@ def stage_names(n_stages):
     return ["self" if s % 2 == 0 else "cross" for s in range(n_stages)]
 
 
-def attentional_gnn(x0, x1, weights, heads, eps, n_stages=None):
+def attentional_gnn(x0, x1, weights, heads, eps, n_stages=None, bidirectional=False):
     """Stages alternate self (A<-A, B<-B) and cross (A<-B, B<-A); both deltas are
     computed from the pre-stage states and then added [realcat notes, section
-    多层GNN, AttentionalGNN]."""
+    多层GNN, AttentionalGNN].  bidirectional=True: the cross stages take their
+    messages from bidirectional_cross_attention (one qk projection, one
+    similarity for both directions [LightGlue review, section 2.3]) and feed
+    them to the same update MLP."""
     stages = weights["stages"]
     if n_stages is None:
         n_stages = len(stages)
     for s, name in enumerate(stage_names(n_stages)):
+        if name == "cross" and bidirectional:
+            st = stages[s]
+            m0, m1 = bidirectional_cross_attention(x0, x1, st, heads)
+            d0 = mlp(np.concatenate([x0, m0], axis=1), [st["W1"], st["W2"]], [st["b1"], st["b2"]], [st["bn1"]], eps)
+            d1 = mlp(np.concatenate([x1, m1], axis=1), [st["W1"], st["W2"]], [st["b1"], st["b2"]], [st["bn1"]], eps)
+            x0, x1 = x0 + d0, x1 + d1
+            continue
         if name == "cross":
             src0, src1 = x1, x0
         else:

@@ -793,3 +793,23 @@ def test_log_sinkhorn_backward_by_finite_differences():
         zp[i, j] += h
         zm[i, j] -= h
         assert abs((loss(zp) - loss(zm)) / (2 * h) - grad[i, j]) < 1e-6
+
+
+def test_bidirectional_gnn_with_tied_projections_is_the_standard_gnn(weights):
+    # with Wk = Wq (and bk = bq) in every cross stage, the bidirectional cross
+    # stages compute the same messages as the standard ones
+    rng = np.random.default_rng(50)
+    x0 = rng.standard_normal((8, 256)) * 0.3
+    x1 = rng.standard_normal((6, 256)) * 0.3
+    w = dict(weights)
+    w["stages"] = [dict(st) for st in weights["stages"][:4]]
+    for st in w["stages"]:
+        st["Wk"], st["bk"] = st["Wq"], st["bq"]
+    a0, a1 = O.attentional_gnn(x0, x1, w, 4, 1e-5, n_stages=4, bidirectional=True)
+    r0, r1 = O.attentional_gnn(x0, x1, w, 4, 1e-5, n_stages=4)
+    np.testing.assert_allclose(a0, r0, rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(a1, r1, rtol=1e-11, atol=1e-12)
+    # and untied projections differ (the bidirectional stage ignores Wk)
+    u0, _ = O.attentional_gnn(x0, x1, weights, 4, 1e-5, n_stages=2, bidirectional=True)
+    s0, _ = O.attentional_gnn(x0, x1, weights, 4, 1e-5, n_stages=2)
+    assert np.abs(u0 - s0).max() > 1e-6
