@@ -105,8 +105,11 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def algorithmic_work(B, M, N, n_stages=18, T=100, D=256):
-    """Per-launch algorithmic work of each kernel class (FLOPs, or bytes for Sinkhorn)."""
+def algorithmic_work(B, M, N, n_stages=18, T=100, D=256, precision="bf16"):
+    """Per-launch algorithmic work of each kernel class (FLOPs, or bytes for Sinkhorn).
+    The fp32 path runs its GEMMs and attention on the FP32 FMA pipes (CUDA cores):
+    those classes are bound by plain ALU arithmetic there."""
+    mm = "tensor" if precision == "bf16" else "alu"
     P = M + N
     R = B * P
     self_pairs = B * (M * M + N * N)
@@ -117,17 +120,23 @@ def algorithmic_work(B, M, N, n_stages=18, T=100, D=256):
     E = (M + 1) * (N + 1)
     return {
         "encoder": ("alu", 2.0 * R * (3 * 32 + 32 * 64 + 64 * 128 + 128 * 256 + 256 * 256)),
-        "qkv_gemm": ("tensor", 2.0 * R * 3 * D * D),
-        "attention": ("tensor", float(attn_flops)),
-        "mlp1_gemm": ("tensor", 2.0 * R * (2 * D) * (2 * D)),
-        "mlp2_gemm": ("tensor", 2.0 * R * D * (2 * D)),
-        "proj_gemm": ("tensor", 2.0 * R * D * D),
-        "score_gemm": ("tensor", 2.0 * B * M * N * D),
+        "qkv_gemm": (mm, 2.0 * R * 3 * D * D),
+        "attention": (mm, float(attn_flops)),
+        "mlp1_gemm": (mm, 2.0 * R * (2 * D) * (2 * D)),
+        "mlp2_gemm": (mm, 2.0 * R * D * (2 * D)),
+        "proj_gemm": (mm, 2.0 * R * D * D),
+        "score_gemm": (mm, 2.0 * B * M * N * D),
         # streamed-byte model of the transport: two fp32 passes over the augmented matrix per iteration
         "sinkhorn": ("hbm", 2.0 * T * 4 * E * B),
         # double-softmax head: the compulsory bytes (read the similarity, write log P)
         "dsm_head": ("hbm", 8.0 * E * B),
     }
+
+
+def fp32_alu_peak_tflops(sm_mhz):
+    """Peak of plain fp32 arithmetic from the unit counts and the clock: 148 SMs x
+    128 FP32 lanes x 2 FLOP (one FMA) per clock."""
+    return 148 * 128 * 2 * (sm_mhz or 1965.0) * 1e6 / 1e12
 
 
 class ClockSampler:
@@ -410,7 +419,8 @@ def run_native(args, w):
 
     # roofline of the dominant kernel class
     peaks, peak_src = load_peaks()
-    work = algorithmic_work(B, M, N)
+    work = algorithmic_work(B, M, N, precision=w.precision)
+    alu_peak = fp32_alu_peak_tflops(clk.get("sm_mhz"))
     dom = max(per_class, key=lambda k: per_class[k][0])
     ms_dom, n_dom = per_class[dom]
     bound, units = work[dom]
@@ -420,12 +430,13 @@ def run_native(args, w):
     elif bound == "tensor":
         achieved, peak, unit = units / avg_s / 1e12, peaks["bf16_tflops"], "TFLOP/s"
     else:
-        achieved, peak, unit = units / avg_s / 1e12, None, "TFLOP/s"
+        achieved, peak, unit = units / avg_s / 1e12, alu_peak, "TFLOP/s"
     traffic, traffic_src = measured_traffic(dom, w.name)
     roofline = {"bound": bound, "kernel": dom, "achieved": achieved, "peak": peak, "unit": unit,
                 "frac": (achieved / peak) if peak else None, "traffic": traffic,
                 "traffic_source": traffic_src,
-                "peak_source": peak_src + (" (burst)" if bound == "tensor" else "")}
+                "peak_source": (peak_src + (" (burst)" if bound == "tensor" else "")) if bound != "alu"
+                else "derived: 148 SMs x 128 FP32 lanes x 2 FLOP x the sampled SM clock"}
     if dom == "sinkhorn":
         # the other bounds of the transport kernel: one ex2 per element and
         # iteration on the MUFU (16 per clock and SM), and the compulsory bytes
@@ -450,6 +461,8 @@ def run_native(args, w):
             rate = {"TFLOP/s": r}
             if b == "tensor":
                 rate["frac_tensor"] = r / peaks["bf16_tflops"]
+            else:
+                rate["frac_alu"] = r / alu_peak
         breakdown[k] = {"ms_per_step": ms / args.steps, "launches_per_step": n // args.steps, **rate}
     gnn = [k for k in ("qkv_gemm", "attention", "mlp1_gemm", "mlp2_gemm", "proj_gemm", "score_gemm")
            if k in per_class]
@@ -458,9 +471,12 @@ def run_native(args, w):
     gnn_events_s = sum(per_class[k][0] for k in gnn) / 1000.0
     gnn_segment = None
     if gnn_s > 0:
+        # the bf16 path against the tensor-core peak, the fp32 path against the FP32 ALU peak
+        gpeak, gname = ((peaks["bf16_tflops"], "frac_tensor") if w.precision == "bf16"
+                        else (alu_peak, "frac_alu"))
         gnn_segment = {"ms_per_step": gnn_s * 1e3 / args.steps, "TFLOP/s": gnn_flops / gnn_s / 1e12,
-                       "frac_tensor": gnn_flops / gnn_s / 1e12 / peaks["bf16_tflops"],
-                       "frac_tensor_per_kernel_events": (gnn_flops / gnn_events_s / 1e12 / peaks["bf16_tflops"])
+                       gname: gnn_flops / gnn_s / 1e12 / gpeak,
+                       gname + "_per_kernel_events": (gnn_flops / gnn_events_s / 1e12 / gpeak)
                        if gnn_events_s > 0 else None,
                        "timing": "one event pair around the chained GNN launches (q|k|v to scores)"}
 
@@ -473,7 +489,7 @@ def run_native(args, w):
         "data": "synthetic (seeded keypoint pairs, random-init weights)",
         "config": _config(w, world, args.head, exit_layer),
         "roofline": roofline,
-        "gnn_tensor_frac": gnn_segment["frac_tensor"] if gnn_segment else None,
+        "gnn_tensor_frac": gnn_segment.get("frac_tensor") if gnn_segment else None,
         "gnn": gnn_segment,
         "kernels": breakdown,
         "kernels_timing": "an event before every launch, which ends the launch overlap: per-kernel "

@@ -64,3 +64,12 @@ def test_planted_exit_weights_make_the_oracle_exit_after_the_layer():
     c = bench._config(synth.WORKLOADS["pair2048"], 1, "sinkhorn", 1)
     assert c["adaptive_depth"]["exit_after_layer"] == 1
     assert "adaptive_depth" not in bench._config(synth.WORKLOADS["pair2048"], 1)
+
+
+def test_fp32_path_is_bounded_by_the_alu_peak():
+    w32 = bench.algorithmic_work(1, 64, 64, precision="fp32")
+    w16 = bench.algorithmic_work(1, 64, 64)
+    for k in ("qkv_gemm", "attention", "mlp1_gemm", "mlp2_gemm", "proj_gemm", "score_gemm"):
+        assert w32[k][0] == "alu" and w16[k][0] == "tensor" and w32[k][1] == w16[k][1]
+    # 148 SMs x 128 FP32 lanes x 2 FLOP at 1965 MHz
+    assert abs(bench.fp32_alu_peak_tflops(1965.0) - 74.45) < 0.01
