@@ -290,6 +290,75 @@ def planted_exit_weights(weights, exit_layer):
     return w
 
 
+def summarize(per_class, per_seg, w, B, M, N, steps, clk, measured_traffic_fn=None):
+    """Roofline of the dominant kernel class, the per-class breakdown and the
+    chained-GNN segment from the timing passes (pure host arithmetic)."""
+    if measured_traffic_fn is None:
+        measured_traffic_fn = measured_traffic
+    peaks, peak_src = load_peaks()
+    work = algorithmic_work(B, M, N, precision=w.precision)
+    alu_peak = fp32_alu_peak_tflops(clk.get("sm_mhz"))
+    dom = max(per_class, key=lambda k: per_class[k][0])
+    ms_dom, n_dom = per_class[dom]
+    bound, units = work[dom]
+    avg_s = ms_dom / n_dom / 1000.0
+    if bound == "hbm":
+        achieved, peak, unit = units / avg_s / 1e9, peaks["hbm_gbs"], "GB/s"
+    elif bound == "tensor":
+        achieved, peak, unit = units / avg_s / 1e12, peaks["bf16_tflops"], "TFLOP/s"
+    else:
+        achieved, peak, unit = units / avg_s / 1e12, alu_peak, "TFLOP/s"
+    traffic, traffic_src = measured_traffic_fn(dom, w.name)
+    roofline = {"bound": bound, "kernel": dom, "achieved": achieved, "peak": peak, "unit": unit,
+                "frac": (achieved / peak) if peak else None, "traffic": traffic,
+                "traffic_source": traffic_src,
+                "peak_source": (peak_src + (" (burst)" if bound == "tensor" else "")) if bound != "alu"
+                else "derived: 148 SMs x 128 FP32 lanes x 2 FLOP x the sampled SM clock"}
+    if dom == "sinkhorn":
+        # the other bounds of the transport kernel: one ex2 per element and
+        # iteration on the MUFU (16 per clock and SM), and the compulsory bytes
+        # (read S, write log P: 8 E)
+        E = (M + 1) * (N + 1) * B
+        sm_clock = (clk.get("sm_mhz") or 1965.0) * 1e6
+        roofline["other_bounds_ms"] = {
+            "mufu_ex2": 100 * E / (148 * 16 * sm_clock) * 1e3,
+            "compulsory_bytes": 8 * E / (peaks["hbm_gbs"] * 1e9) * 1e3,
+            "kernel": avg_s * 1e3,
+        }
+    breakdown = {}
+    for k, (ms, n) in per_class.items():
+        if n == 0:
+            continue
+        b, u = work[k]
+        avg = ms / n / 1000.0
+        if b == "hbm":
+            rate = {"GB/s": u / avg / 1e9, "frac_hbm": u / avg / 1e9 / peaks["hbm_gbs"]}
+        else:
+            r = u / avg / 1e12
+            rate = {"TFLOP/s": r}
+            if b == "tensor":
+                rate["frac_tensor"] = r / peaks["bf16_tflops"]
+            else:
+                rate["frac_alu"] = r / alu_peak
+        breakdown[k] = {"ms_per_step": ms / steps, "launches_per_step": n // steps, **rate}
+    gnn = [k for k in ("qkv_gemm", "attention", "mlp1_gemm", "mlp2_gemm", "proj_gemm", "score_gemm")
+           if k in per_class]
+    gnn_flops = sum(work[k][1] * per_class[k][1] for k in gnn)
+    gnn_s = per_seg.get("gnn", (0.0, 0))[0] / 1000.0
+    gnn_events_s = sum(per_class[k][0] for k in gnn) / 1000.0
+    gnn_segment = None
+    if gnn_s > 0:
+        # the bf16 path against the tensor-core peak, the fp32 path against the FP32 ALU peak
+        gpeak, gname = ((peaks["bf16_tflops"], "frac_tensor") if w.precision == "bf16"
+                        else (alu_peak, "frac_alu"))
+        gnn_segment = {"ms_per_step": gnn_s * 1e3 / steps, "TFLOP/s": gnn_flops / gnn_s / 1e12,
+                       gname: gnn_flops / gnn_s / 1e12 / gpeak,
+                       gname + "_per_kernel_events": (gnn_flops / gnn_events_s / 1e12 / gpeak)
+                       if gnn_events_s > 0 else None,
+                       "timing": "one event pair around the chained GNN launches (q|k|v to scores)"}
+    return roofline, breakdown, gnn_segment
+
+
 def run_native(args, w):
     import torch
     import torch.distributed as dist
@@ -417,68 +486,7 @@ def run_native(args, w):
     h2d = sum(v.numel() * v.element_size() for v in host.values())
     d2h = sum(v.numel() * v.element_size() for v in (hm0, hm1, hs0, hs1))
 
-    # roofline of the dominant kernel class
-    peaks, peak_src = load_peaks()
-    work = algorithmic_work(B, M, N, precision=w.precision)
-    alu_peak = fp32_alu_peak_tflops(clk.get("sm_mhz"))
-    dom = max(per_class, key=lambda k: per_class[k][0])
-    ms_dom, n_dom = per_class[dom]
-    bound, units = work[dom]
-    avg_s = ms_dom / n_dom / 1000.0
-    if bound == "hbm":
-        achieved, peak, unit = units / avg_s / 1e9, peaks["hbm_gbs"], "GB/s"
-    elif bound == "tensor":
-        achieved, peak, unit = units / avg_s / 1e12, peaks["bf16_tflops"], "TFLOP/s"
-    else:
-        achieved, peak, unit = units / avg_s / 1e12, alu_peak, "TFLOP/s"
-    traffic, traffic_src = measured_traffic(dom, w.name)
-    roofline = {"bound": bound, "kernel": dom, "achieved": achieved, "peak": peak, "unit": unit,
-                "frac": (achieved / peak) if peak else None, "traffic": traffic,
-                "traffic_source": traffic_src,
-                "peak_source": (peak_src + (" (burst)" if bound == "tensor" else "")) if bound != "alu"
-                else "derived: 148 SMs x 128 FP32 lanes x 2 FLOP x the sampled SM clock"}
-    if dom == "sinkhorn":
-        # the other bounds of the transport kernel: one ex2 per element and
-        # iteration on the MUFU (16 per clock and SM), and the compulsory bytes
-        # (read S, write log P: 8 E)
-        E = (M + 1) * (N + 1) * B
-        sm_clock = (clk.get("sm_mhz") or 1965.0) * 1e6
-        roofline["other_bounds_ms"] = {
-            "mufu_ex2": 100 * E / (148 * 16 * sm_clock) * 1e3,
-            "compulsory_bytes": 8 * E / (peaks["hbm_gbs"] * 1e9) * 1e3,
-            "kernel": avg_s * 1e3,
-        }
-    breakdown = {}
-    for k, (ms, n) in per_class.items():
-        if n == 0:
-            continue
-        b, u = work[k]
-        avg = ms / n / 1000.0
-        if b == "hbm":
-            rate = {"GB/s": u / avg / 1e9, "frac_hbm": u / avg / 1e9 / peaks["hbm_gbs"]}
-        else:
-            r = u / avg / 1e12
-            rate = {"TFLOP/s": r}
-            if b == "tensor":
-                rate["frac_tensor"] = r / peaks["bf16_tflops"]
-            else:
-                rate["frac_alu"] = r / alu_peak
-        breakdown[k] = {"ms_per_step": ms / args.steps, "launches_per_step": n // args.steps, **rate}
-    gnn = [k for k in ("qkv_gemm", "attention", "mlp1_gemm", "mlp2_gemm", "proj_gemm", "score_gemm")
-           if k in per_class]
-    gnn_flops = sum(work[k][1] * per_class[k][1] for k in gnn)
-    gnn_s = per_seg.get("gnn", (0.0, 0))[0] / 1000.0
-    gnn_events_s = sum(per_class[k][0] for k in gnn) / 1000.0
-    gnn_segment = None
-    if gnn_s > 0:
-        # the bf16 path against the tensor-core peak, the fp32 path against the FP32 ALU peak
-        gpeak, gname = ((peaks["bf16_tflops"], "frac_tensor") if w.precision == "bf16"
-                        else (alu_peak, "frac_alu"))
-        gnn_segment = {"ms_per_step": gnn_s * 1e3 / args.steps, "TFLOP/s": gnn_flops / gnn_s / 1e12,
-                       gname: gnn_flops / gnn_s / 1e12 / gpeak,
-                       gname + "_per_kernel_events": (gnn_flops / gnn_events_s / 1e12 / gpeak)
-                       if gnn_events_s > 0 else None,
-                       "timing": "one event pair around the chained GNN launches (q|k|v to scores)"}
+    roofline, breakdown, gnn_segment = summarize(per_class, per_seg, w, B, M, N, args.steps, clk)
 
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,

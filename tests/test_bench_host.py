@@ -73,3 +73,52 @@ def test_fp32_path_is_bounded_by_the_alu_peak():
         assert w32[k][0] == "alu" and w16[k][0] == "tensor" and w32[k][1] == w16[k][1]
     # 148 SMs x 128 FP32 lanes x 2 FLOP at 1965 MHz
     assert abs(bench.fp32_alu_peak_tflops(1965.0) - 74.45) < 0.01
+
+
+def _fake_classes(steps, sinkhorn_ms, gnn_ms):
+    per_class = {"encoder": (0.06 * steps, steps), "qkv_gemm": (0.18 * steps, 18 * steps),
+                 "attention": (0.41 * steps, 18 * steps), "mlp1_gemm": (0.22 * steps, 18 * steps),
+                 "mlp2_gemm": (0.22 * steps, 18 * steps), "proj_gemm": (0.01 * steps, steps),
+                 "score_gemm": (0.012 * steps, steps), "sinkhorn": (sinkhorn_ms * steps, steps),
+                 "gnn": (0.0, 0)}
+    per_seg = {"encoder": (0.06 * steps, steps), "gnn": (gnn_ms * steps, steps),
+               "sinkhorn": (sinkhorn_ms * steps, steps)}
+    return per_class, per_seg
+
+
+def test_summarize_bf16_pair2048():
+    from learned_sparse_feature_b200 import synth
+    w = synth.WORKLOADS["pair2048"]
+    per_class, per_seg = _fake_classes(20, 0.70, 0.65)
+    roof, breakdown, gnn = bench.summarize(per_class, per_seg, w, 1, 2048, 2048, 20, {"sm_mhz": 1965.0},
+                                           measured_traffic_fn=lambda k, n: (None, None))
+    assert roof["kernel"] == "sinkhorn" and roof["bound"] == "hbm" and 0.5 < roof["frac"] < 1.0
+    assert set(roof["other_bounds_ms"]) == {"mufu_ex2", "compulsory_bytes", "kernel"}
+    assert "gnn" not in breakdown and breakdown["attention"]["launches_per_step"] == 18
+    assert "frac_tensor" in breakdown["attention"] and "frac_alu" in breakdown["encoder"]
+    assert abs(gnn["ms_per_step"] - 0.65) < 1e-12 and 0.1 < gnn["frac_tensor"] < 0.5
+
+
+def test_summarize_fp32_reports_alu_fractions():
+    from learned_sparse_feature_b200 import synth
+    w = synth.WORKLOADS["pair64_fp32"]
+    per_class, per_seg = _fake_classes(20, 0.34, 2.29)
+    per_class["mlp2_gemm"] = (0.92 * 20, 18 * 20)       # the largest class on this path
+    roof, breakdown, gnn = bench.summarize(per_class, per_seg, w, 1, 64, 64, 20, {"sm_mhz": None},
+                                           measured_traffic_fn=lambda k, n: (None, None))
+    assert roof["kernel"] == "mlp2_gemm" and roof["bound"] == "alu"
+    assert roof["peak"] == bench.fp32_alu_peak_tflops(1965.0) and roof["peak_source"].startswith("derived")
+    assert "frac_alu" in breakdown["mlp1_gemm"] and "frac_tensor" not in breakdown["mlp1_gemm"]
+    assert "frac_alu" in gnn and "frac_tensor" not in gnn
+
+
+def test_summarize_double_softmax_head_class():
+    from learned_sparse_feature_b200 import synth
+    w = synth.WORKLOADS["pair2048"]
+    per_class, per_seg = _fake_classes(20, 0.70, 0.65)
+    per_class["dsm_head"] = per_class.pop("sinkhorn")
+    per_class["dsm_head"] = (0.115 * 20, 20 * 20)
+    roof, breakdown, _ = bench.summarize(per_class, per_seg, w, 1, 2048, 2048, 20, {"sm_mhz": 1965.0},
+                                         measured_traffic_fn=lambda k, n: (None, None))
+    assert roof["kernel"] == "attention" and roof["bound"] == "tensor"
+    assert "frac_hbm" in breakdown["dsm_head"]
