@@ -471,7 +471,9 @@ def attentional_gnn_adaptive(xs0, xs1, weights, heads, eps, depth_confidence, n_
     num_points = sum(len(x) for x in xs0) + sum(len(x) for x in xs1)
     for layer in range(n_layers):
         if any(len(x) == 0 for x in xs0) or any(len(x) == 0 for x in xs1):
-            break                                # a pair without points left: no more layers
+            # a pair without points left: no more layers (reading: the count
+            # reported is the layers that ran)
+            return xs0, xs1, kept0, kept1, layer
         for s in (2 * layer, 2 * layer + 1):
             for b in range(len(xs0)):
                 x0, x1 = xs0[b], xs1[b]

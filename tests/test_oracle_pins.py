@@ -813,3 +813,21 @@ def test_bidirectional_gnn_with_tied_projections_is_the_standard_gnn(weights):
     u0, _ = O.attentional_gnn(x0, x1, weights, 4, 1e-5, n_stages=2, bidirectional=True)
     s0, _ = O.attentional_gnn(x0, x1, weights, 4, 1e-5, n_stages=2)
     assert np.abs(u0 - s0).max() > 1e-6
+
+
+def test_pruning_every_point_of_an_image_ends_the_layers(weights):
+    # matchability 0 everywhere and no exit classifier: after layer 0 every
+    # point is pruned, the next layer does not run and nothing is matched
+    rng = np.random.default_rng(22)
+    pairs = [synth.make_pair(rng, 6, 5, 0.5)]
+    batch = {k: np.stack([p[k] for p in pairs]) for k in ("kpts0", "conf0", "desc0", "kpts1", "conf1", "desc1")}
+    w = dict(weights)
+    w["mt_w"] = [np.zeros(256)] * 9
+    w["mt_b"] = [-50.0] * 9
+    out, layers = O.superglue_batch_adaptive(batch, w, None, n_stages=6, width_confidence=0.99,
+                                             pruning_threshold=0)
+    assert layers == 1                           # only layer 0 ran
+    res = out[0]
+    assert len(res["kept0"]) == 0 and len(res["kept1"]) == 0 and res["log_P"] is None
+    assert np.all(res["matches0"] == -1) and np.all(res["matches1"] == -1)
+    assert np.all(res["mscores0"] == 0) and np.all(res["mscores1"] == 0)
