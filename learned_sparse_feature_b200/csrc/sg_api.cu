@@ -418,7 +418,7 @@ cudaError_t run_network(sg_handle* h, int B, int M, int N, const Inputs& in, flo
 cudaError_t run_transport(sg_handle* h, int B, int M, int N, const float* S, long long lds,
                           long long strideS, float* logP, int32_t* m0, int32_t* m1, float* s0,
                           float* s1, cudaStream_t st, int* launches) {
-  const size_t C = N + 1, R = M + 1;
+  const size_t R = M + 1;
   unsigned char* p = h->sk_scratch;
   SinkhornArgs a{};
   a.barrier = reinterpret_cast<unsigned*>(p);
