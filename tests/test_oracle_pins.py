@@ -831,3 +831,19 @@ def test_pruning_every_point_of_an_image_ends_the_layers(weights):
     assert len(res["kept0"]) == 0 and len(res["kept1"]) == 0 and res["log_P"] is None
     assert np.all(res["matches0"] == -1) and np.all(res["matches1"] == -1)
     assert np.all(res["mscores0"] == 0) and np.all(res["mscores1"] == 0)
+
+
+def test_batch_adaptive_without_exit_or_pruning_is_the_pair_pass(weights):
+    # the batch driver (encoder, lockstep layers, head, map back) reduces to
+    # superglue_pair for every pair when nothing exits and nothing is pruned
+    rng = np.random.default_rng(23)
+    pairs = [synth.make_pair(rng, 10, 8, 0.5) for _ in range(2)]
+    batch = {k: np.stack([p[k] for p in pairs]) for k in ("kpts0", "conf0", "desc0", "kpts1", "conf1", "desc1")}
+    out, layers = O.superglue_batch_adaptive(batch, weights, None, n_stages=4)
+    assert layers == 2
+    for b in range(2):
+        ref = O.superglue_pair(*(batch[k][b] for k in ("kpts0", "conf0", "desc0", "kpts1", "conf1", "desc1")),
+                               weights, n_stages=4)
+        np.testing.assert_array_equal(out[b]["log_P"], ref["log_P"])
+        for k in ("matches0", "matches1", "mscores0", "mscores1"):
+            np.testing.assert_array_equal(out[b][k], ref[k])
